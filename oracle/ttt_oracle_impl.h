@@ -27,7 +27,8 @@
  *    mini-batch started from; the running state W_t subtracts the gradients of
  *    all tokens s <= t of the mini-batch, each times its own eta_s, and the
  *    output of token t uses that W_t.  b = 1 is the per-token rule [LR1];
- *    b = T is batch GD [LR3].
+ *    b = T is batch GD [LR3].  When b does not divide T, the last mini-batch
+ *    holds the remaining T mod b tokens.
  *  - LayerNorm: over the d features of one token, biased variance, eps inside
  *    the square root; gamma and beta are fixed (outer-loop) parameters, the
  *    inner loop updates W and b only.
@@ -154,7 +155,7 @@ int FN(oracle_ttt_linear)(int B, int H, int T, int d, int mb, int mode, REAL eps
                           const REAL* Q, const REAL* K, const REAL* V, const REAL* eta,
                           const REAL* W0, const REAL* b0, const REAL* gamma,
                           const REAL* beta, REAL* Z, REAL* W_T, REAL* b_T, int nthreads) {
-    if (B < 0 || H < 0 || T < 0 || d <= 0 || mb <= 0 || (T % mb) != 0) return -1;
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || mb <= 0) return -1;
     if (mode != ORACLE_MODE_PLAIN && mode != ORACLE_MODE_LN_RESIDUAL) return -1;
     if (nthreads <= 0) nthreads = 1;
     long nbh = (long)B * H;
@@ -172,7 +173,7 @@ int FN(oracle_ttt_linear)(int B, int H, int T, int d, int mb, int mode, REAL eps
         for (int m = 0; m < T; m += mb) {
             memcpy(Wc, Ws, sizeof(REAL) * (size_t)d * d);
             memcpy(bc, bs, sizeof(REAL) * d);
-            for (int t = m; t < m + mb; t++) {
+            for (int t = m; t < m + mb && t < T; t++) {
                 long row = (bh * T + t) * d;
                 REAL e = eta[bh * T + t];
                 /* gradient of token t, taken at the mini-batch's start state */
@@ -278,7 +279,7 @@ int FN(oracle_ttt_mlp)(int B, int H, int T, int d, int hid, int mb, REAL eps, co
                        const REAL* b1_0, const REAL* W2_0, const REAL* b2_0, const REAL* gamma,
                        const REAL* beta, REAL* Z, REAL* W1_T, REAL* b1_T, REAL* W2_T,
                        REAL* b2_T, int nthreads) {
-    if (B < 0 || H < 0 || T < 0 || d <= 0 || hid <= 0 || mb <= 0 || (T % mb) != 0) return -1;
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || hid <= 0 || mb <= 0) return -1;
     if (nthreads <= 0) nthreads = 1;
     long nbh = (long)B * H;
     size_t nW = (size_t)d * hid;
@@ -301,7 +302,7 @@ int FN(oracle_ttt_mlp)(int B, int H, int T, int d, int hid, int mb, REAL eps, co
             memcpy(W2c, W2s, sizeof(REAL) * nW);
             memcpy(b1c, b1s, sizeof(REAL) * hid);
             memcpy(b2c, b2s, sizeof(REAL) * d);
-            for (int t = m; t < m + mb; t++) {
+            for (int t = m; t < m + mb && t < T; t++) {
                 long row = (bh * T + t) * d;
                 REAL e = eta[bh * T + t];
                 FN(mlp_token_grads)(d, hid, eps, K + row, V + row, W1s, b1s, W2s, b2s, gam, bet,

@@ -72,7 +72,7 @@ def minibatch_restatement(fn, params, Q, K, V, eta, mb):
     Z = torch.zeros_like(Q)
     for m in range(0, T, mb):
         cur = [p.clone() for p in start]
-        for t in range(m, m + mb):
+        for t in range(m, min(m + mb, T)):
             _, gs = autograd_grads(fn, start, K[t], V[t])
             cur = [c - eta[t] * g for c, g in zip(cur, gs)]
             Z[t] = fn(Q[t], *cur)
@@ -260,9 +260,11 @@ def test_b1_equals_online_gd(mode):
     assert rel(W_T[0, 0], W.numpy()) < 1e-11
 
 
-@pytest.mark.parametrize("mode,mb", [(LN, 8), (LN, 16), (PLAIN, 8), (LN, 48)])
-def test_minibatch_rule_linear(mode, mb):
-    Q, K, V, eta, W0, b0, gamma, beta = small_linear_case(5, T=48, mode=mode)
+@pytest.mark.parametrize("mode,mb,T", [(LN, 8, 48), (LN, 16, 48), (PLAIN, 8, 48), (LN, 48, 48),
+                                       (LN, 16, 43), (PLAIN, 16, 21)])
+def test_minibatch_rule_linear(mode, mb, T):
+    """Includes ragged T: the last mini-batch holds the remaining T mod b tokens."""
+    Q, K, V, eta, W0, b0, gamma, beta = small_linear_case(5, T=T, mode=mode)
     Z, W_T, b_T = oracle.ttt_linear(Q, K, V, eta, W0, b0, gamma, beta, mb, mode)
     g, bt = t64(gamma[0]), t64(beta[0])
     fn = lambda x, W_, b_: f_linear(x, W_, b_, g, bt, mode)
@@ -275,9 +277,9 @@ def test_minibatch_rule_linear(mode, mb):
         assert rel(b_T[0, 0], b_ref.numpy()) < 1e-11
 
 
-@pytest.mark.parametrize("mb", [1, 8])
-def test_minibatch_rule_mlp(mb):
-    Q, K, V, eta, W1, b1, W2, b2, gamma, beta = small_mlp_case(9, T=24)
+@pytest.mark.parametrize("mb,T", [(1, 24), (8, 24), (16, 27)])
+def test_minibatch_rule_mlp(mb, T):
+    Q, K, V, eta, W1, b1, W2, b2, gamma, beta = small_mlp_case(9, T=T)
     Z, W1_T, b1_T, W2_T, b2_T = oracle.ttt_mlp(Q, K, V, eta, W1, b1, W2, b2, gamma, beta, mb)
     g, bt = t64(gamma[0]), t64(beta[0])
     fn = lambda x, a, b_, c, e: f_mlp(x, a, b_, c, e, g, bt)
@@ -521,8 +523,8 @@ def _run_pins_with(lib_path):
         lambda: test_mlp_gradient_autograd(),
         lambda: test_mlp_gradient_finite_differences(0),
         lambda: test_b1_equals_online_gd(LN),
-        lambda: test_minibatch_rule_linear(LN, 8),
-        lambda: test_minibatch_rule_mlp(8),
+        lambda: test_minibatch_rule_linear(LN, 8, 48),
+        lambda: test_minibatch_rule_mlp(8, 24),
     ]
     try:
         for pin in pins:
