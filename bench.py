@@ -1,0 +1,346 @@
+#!/usr/bin/env python
+"""Forward tokens/s of the TTT-Linear scan on B200 (1.3B-layer shape, 32k context).
+
+One step = one ttt_linear_forward call over the whole workload
+(B=2, H=32, T=32768, d=64, b=16, bf16 Q/K/V, fp32 state), inputs resident in
+HBM.  tokens/s = B*T / step time (all H heads).  The inputs (1.35 GB per
+step) are larger than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own instance of the workload (the
+(batch, head) scans are independent; no collective on the data path), so
+scaling is weak and value = all ranks' tokens / max-over-ranks time.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from test_sequence_layers_ttt_b200.inputs import WORKLOADS, make_inputs, select_heads  # noqa: E402
+
+METRIC = "TTT forward tokens/sec on 1 B200 (1.3B-layer shape, 32k ctx); % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+KEYS = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+
+
+def algorithmic_bytes(w) -> int:
+    """Bytes the scan must move: Q/K/V, eta, Z per head-token, the state read
+    once and written once per (batch, head), gamma/beta once."""
+    es = 2 if w.dtype == "bf16" else 4
+    per_tok = 3 * w.d * es + 4 + 4 * w.d
+    state = 2 * (w.d * w.d + w.d) * 4
+    return w.head_tokens * per_tok + w.B * w.H * state + 2 * w.H * w.d * 4
+
+
+def algorithmic_flops(w) -> int:
+    """6 d^2 (X W, Q W, update) + 4*16*d (Q X^T, A G) per head-token."""
+    return w.head_tokens * (6 * w.d * w.d + 4 * 16 * w.d)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "test_sequence_layers_ttt_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    entry = rec.get(f"{kernel}:{workload}")
+    if not entry or entry.get("source_hash") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(w, inp, target_s: float):
+    """Time the float64 oracle (all host cores) on whole (batch, head) scans of
+    the workload, as many as fit in about target_s seconds; returns tokens/s in
+    the workload's unit (B*T tokens cover all H heads)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    B, H = inp["Q"].shape[:2]
+    pairs_all = [(b, h) for b in range(B) for h in range(H)]
+    # calibrate on one scan
+    sel = select_heads(inp, pairs_all[:1])
+    t0 = time.perf_counter()
+    oracle.ttt_linear(*(sel[k] for k in KEYS), w.mini_batch, w.mode, w.ln_eps, threads=1)
+    one = time.perf_counter() - t0
+    n = max(1, min(len(pairs_all), int(target_s / max(one, 1e-6) * min(cores, len(pairs_all)))))
+    n = max(min(n, len(pairs_all)), 1)
+    sel = select_heads(inp, pairs_all[:n])
+    t0 = time.perf_counter()
+    oracle.ttt_linear(*(sel[k] for k in KEYS), w.mini_batch, w.mode, w.ln_eps, threads=cores)
+    dt = time.perf_counter() - t0
+    tokens = n * w.T / w.H
+    used = min(cores, n)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{n} of {w.B * w.H} (batch, head) scans at full T={w.T}, float64 primal oracle, "
+                      f"{dt:.2f} s; tokens counted as scans*T/H"}
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    inp = make_inputs(w, args.seed)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, inp, 0.5)
+    vals, samples = [], None
+    t_start = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_oracle_sample(w, inp, args.ref_seconds)
+        vals.append(r["value"])
+        samples = r
+    elapsed = time.perf_counter() - t_start
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": samples["cores"],
+                         "kind": "oracle", "sample": samples["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "mini_batch": w.mini_batch,
+            "qkv_dtype": w.dtype, "state_dtype": "f32", "inner_model": "x + LN(xW + b)",
+            "l2": "inputs (Q/K/V/eta) larger than the 126 MB L2; no flush"}
+
+
+def run_ours(args, world, rank, local):
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    host = make_inputs(w, args.seed + rank)
+    g = {k: v.to(dev) for k, v in host.items()}
+    Z = torch.empty((w.B, w.H, w.T, w.d), dtype=torch.float32, device=dev)
+    W_T = torch.empty_like(g["W0"])
+    b_T = torch.empty_like(g["b0"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ttt.ttt_linear_forward(*(g[k] for k in KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps,
+                               impl=args.kernel, Z=Z, W_T=W_T, b_T=b_T, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)  # let the sampler start
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    total_ms = start.elapsed_time(end)
+    per_launch_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = dist_max(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    kernel_ms = statistics.mean(per_launch_ms)
+    tokens_per_step = w.B * w.T * world
+    value = tokens_per_step / (ms_per_step * 1e-3)
+
+    # end to end through the public API with pinned host buffers
+    host_in = {k: v.pin_memory() for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = (Z.numel() + W_T.numel() + b_T.numel()) * 4
+    ttt.ttt_linear_forward(*(host_in[k] for k in KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    e2e_steps = max(1, min(args.steps, 3))
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        ttt.ttt_linear_forward(*(host_in[k] for k in KEYS), mini_batch=w.mini_batch,
+                               ln_eps=w.ln_eps)  # returns after the device->host copies finish
+    e2e_s = dist_max((time.perf_counter() - t0) / e2e_steps, world)
+    e2e_value = tokens_per_step / e2e_s
+
+    cpu_base = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_sample(w, host, args.ref_seconds)
+
+    if rank == 0:
+        hbm, peak_kind = load_peaks()
+        ab = algorithmic_bytes(w)
+        achieved = ab / (kernel_ms * 1e-3) / 1e9
+        kname = "ttt_linear_tc_kernel" if args.kernel != "generic" else "ttt_linear_generic_kernel"
+        traffic = recorded_traffic(kname, w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(w),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms,
+                         "kernel": kname},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "kernel_impl": args.kernel,
+            "tflops_achieved": algorithmic_flops(w) / (kernel_ms * 1e-3) / 1e12,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="linear_1p3b_32k",
+                    choices=[k for k, v in WORKLOADS.items() if v.kind == "linear"])
+    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore"], default="auto")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-seconds", type=float, default=10.0,
+                    help="CPU seconds of oracle work per reference sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

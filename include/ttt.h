@@ -1,0 +1,150 @@
+/*
+ * ttt.h -- C ABI of the B200 (sm_100a) TTT forward-scan library (libttt_b200.so).
+ *
+ * The library computes the causal forward scan of a Test-Time-Training layer
+ * ("Learning to (Learn at Test Time): RNNs with Expressive Hidden States").
+ * Every (batch, head) pair carries a hidden state that is itself a model f
+ * with weights W.  Over the sequence, in mini-batches of b tokens, the scan
+ * takes gradient steps on the reconstruction loss
+ *     l(W; t) = || f(K_t; W) - V_t ||^2            (sum of squares)
+ * with a per-token learning rate eta_t, and emits z_t = f(Q_t; W_t).
+ *   - State, update rule and output rule: literature record of the paper
+ *     (dmarx.github.io lit-801), Key takeaways, bullet 1.
+ *   - Inner loss and the token-dependent learning rate: same record, bullet 2.
+ *   - Mini-batch updates (b = 16) and LayerNorm + residual inside f: bullet 5.
+ *   - Theorem 1 (linear f, batch GD, eta = 1/2, W0 = 0 is causal linear
+ *     attention): bullet 3.  TTT_PLAIN mode is that linear f.
+ *   - TTT-Linear and TTT-MLP hidden states: the paper's abstract
+ *     (codewithpapers.app record).
+ *
+ * Mini-batch rule: inside a mini-batch every token's gradient is taken at the
+ * state the mini-batch started from; the state used for the output of token t
+ * subtracts eta_s * grad_s for every token s <= t of the mini-batch (t
+ * included).  At the end of the mini-batch that state becomes the next start
+ * state.  If b does not divide T, the last mini-batch holds T mod b tokens.
+ *
+ * Inner models (row vectors, W stored [in][out] row-major):
+ *   TTT_LN_RESIDUAL  f(x) = x + LN(x W + b)
+ *   TTT_PLAIN        f(x) = x W              (no bias, no LN, no residual)
+ *   TTT-MLP          f(x) = x + LN(GELU(x W1 + b1) W2 + b2)
+ * LN(y) = gamma * (y - mean(y)) / sqrt(var(y) + eps) + beta over the d features
+ * of one token, biased variance.  gamma and beta are fixed; the scan updates
+ * W and b (W1, b1, W2, b2 for the MLP).  GELU is the tanh form
+ * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+ *
+ * Conventions shared by every entry point
+ *   Memory      All data pointers are DEVICE pointers on the current CUDA
+ *               device, owned by the caller.  The library allocates no memory
+ *               and keeps no state between calls.
+ *   Layout      Q, K, V, Z: [B][H][T][d] contiguous.  eta: [B][H][T] fp32.
+ *               Per-(batch, head) state: W [B][H][d_in][d_out] fp32, b [B][H][d_out].
+ *               gamma, beta: [H][d] fp32, shared by all batch rows.
+ *   Types       Q, K, V are bf16 (TTT_BF16) or fp32 (TTT_F32); everything else
+ *               is fp32, and the state is carried in fp32.  Z is fp32.
+ *   Alignment   Every pointer must be 16-byte aligned (TTT_ERR_ALIGN).
+ *   Aliasing    W_T may be the same pointer as W0 (and b_T as b0) for an
+ *               in-place state update; any other overlap between an output
+ *               (Z, W_T, b_T) and any other buffer is TTT_ERR_ALIAS.
+ *   Shapes      B, H >= 1; T >= 0 (T = 0 copies the state); mini_batch >= 1
+ *               and either a multiple of 16 or one of 1, 2, 4, 8.
+ *   Stream      Work is enqueued on `stream` (0 = legacy default stream); the
+ *               call does not synchronise.
+ *   Errors      Argument errors are detected on the host before anything is
+ *               launched, and return without side effects.  A launch failure
+ *               returns TTT_ERR_CUDA (from cudaPeekAtLastError).  With the
+ *               environment variable TTT_CHECK=1 the call synchronises the
+ *               stream after the launch and returns TTT_ERR_CUDA on an
+ *               asynchronous error, or TTT_ERR_TIMEOUT if a kernel abandoned a
+ *               bounded wait (its outputs are then undefined).
+ *   Threads     Entry points are re-entrant.
+ *   Continuation  Feeding W_T (b_T) back as W0 (b0) continues the sequence
+ *               exactly when the split falls on a mini-batch boundary.
+ */
+#ifndef TTT_B200_TTT_H
+#define TTT_B200_TTT_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st* ttt_stream_t;
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_NULL = 1,        /* a required pointer is NULL                         */
+    TTT_ERR_SHAPE = 2,       /* B, H, T, mini_batch out of range                   */
+    TTT_ERR_DTYPE = 3,       /* unknown ttt_dtype                                  */
+    TTT_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                   */
+    TTT_ERR_ALIAS = 5,       /* an output overlaps an input other than as allowed  */
+    TTT_ERR_UNSUPPORTED = 6, /* d, hidden, mode or implementation not built       */
+    TTT_ERR_CUDA = 7,        /* CUDA launch or execution error                     */
+    TTT_ERR_TIMEOUT = 8      /* a kernel gave up a bounded wait (TTT_CHECK=1 only) */
+} ttt_status;
+
+typedef enum { TTT_BF16 = 0, TTT_F32 = 1 } ttt_dtype;
+
+typedef enum { TTT_LN_RESIDUAL = 0, TTT_PLAIN = 1 } ttt_mode;
+
+/* Kernel family.  TTT_IMPL_AUTO picks the fastest one built for the shape. */
+typedef enum {
+    TTT_IMPL_AUTO = 0,
+    TTT_IMPL_GENERIC = 1,    /* fp32 SIMT scan: every supported shape, dtype and mode */
+    TTT_IMPL_TENSORCORE = 2  /* tensor-core scan: bf16 Q/K/V, d = 64, LN mode, b = 16  */
+} ttt_impl;
+
+/*
+ * TTT-Linear forward scan.
+ *   d          head dimension: 16, 32 or 64 (TTT_ERR_UNSUPPORTED otherwise)
+ *   mini_batch b of the mini-batch rule above
+ *   qkv_dtype  element type of Q, K, V
+ *   mode       TTT_LN_RESIDUAL or TTT_PLAIN
+ *   ln_eps     LayerNorm epsilon (> 0 in LN mode)
+ *   Q, K, V    [B][H][T][d]
+ *   eta        [B][H][T] per-token inner learning rate
+ *   W0, b0     initial state [B][H][d][d], [B][H][d]; b0 may be NULL in TTT_PLAIN
+ *   ln_gamma, ln_beta  [H][d]; may be NULL in TTT_PLAIN
+ *   Z          [B][H][T][d] fp32 output z_t
+ *   W_T, b_T   final state (same shapes as W0, b0); b_T may be NULL in TTT_PLAIN
+ */
+ttt_status ttt_linear_forward(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                              ttt_mode mode, float ln_eps, const void* Q, const void* K,
+                              const void* V, const float* eta, const float* W0,
+                              const float* b0, const float* ln_gamma, const float* ln_beta,
+                              float* Z, float* W_T, float* b_T, ttt_stream_t stream);
+
+/* As ttt_linear_forward, with an explicit kernel family (TTT_ERR_UNSUPPORTED if
+ * that family does not cover the arguments). */
+ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch,
+                                   ttt_dtype qkv_dtype, ttt_mode mode, float ln_eps,
+                                   const void* Q, const void* K, const void* V,
+                                   const float* eta, const float* W0, const float* b0,
+                                   const float* ln_gamma, const float* ln_beta, float* Z,
+                                   float* W_T, float* b_T, ttt_impl impl, ttt_stream_t stream);
+
+/*
+ * TTT-MLP forward scan, f(x) = x + LN(GELU(x W1 + b1) W2 + b2).
+ *   d = 64 and hidden = 256 are built (TTT_ERR_UNSUPPORTED otherwise).
+ *   W1_0 [B][H][d][hidden], b1_0 [B][H][hidden], W2_0 [B][H][hidden][d], b2_0 [B][H][d]
+ *   W1_T, b1_T, W2_T, b2_T: final state, same shapes; each may be the same
+ *   pointer as its initial-state counterpart.  When mini_batch > 16, W1_T and
+ *   W2_T also hold the mini-batch start state while the scan runs.
+ */
+ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batch,
+                           ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
+                           const void* V, const float* eta, const float* W1_0,
+                           const float* b1_0, const float* W2_0, const float* b2_0,
+                           const float* ln_gamma, const float* ln_beta, float* Z, float* W1_T,
+                           float* b1_T, float* W2_T, float* b2_T, ttt_stream_t stream);
+
+/* Static string naming a status code; never NULL. */
+const char* ttt_status_string(ttt_status status);
+
+/* ABI version of the library (major * 100 + minor). */
+int ttt_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_B200_TTT_H */

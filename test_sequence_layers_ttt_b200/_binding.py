@@ -1,0 +1,180 @@
+"""ctypes binding of libttt_b200.so (include/ttt.h).  Argument marshalling only.
+
+Every step of the scan runs in the library's CUDA kernels; this module checks
+tensor metadata, allocates outputs through torch when the caller does not pass
+them, and forwards raw pointers and the current CUDA stream.  If the inputs
+are CPU tensors, the call copies them to the GPU (from pinned memory), runs
+the kernels and copies the outputs back: the end-to-end path.
+
+Importing this module raises if the library has not been built: there is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
+
+TTT_BF16, TTT_F32 = 0, 1
+TTT_LN_RESIDUAL, TTT_PLAIN = 0, 1
+IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2}
+STATUS = ["TTT_OK", "TTT_ERR_NULL", "TTT_ERR_SHAPE", "TTT_ERR_DTYPE", "TTT_ERR_ALIGN",
+          "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT"]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m test_sequence_layers_ttt_b200.build or __graft_entry__.build())")
+
+lib = ctypes.CDLL(LIB_PATH)
+_I, _F, _P = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+lib.ttt_linear_forward.restype = _I
+lib.ttt_linear_forward.argtypes = [_I] * 7 + [_F] + [_P] * 11 + [_P]
+lib.ttt_linear_forward_impl.restype = _I
+lib.ttt_linear_forward_impl.argtypes = [_I] * 7 + [_F] + [_P] * 11 + [_I, _P]
+lib.ttt_mlp_forward.restype = _I
+lib.ttt_mlp_forward.argtypes = [_I] * 7 + [_F] + [_P] * 15 + [_P]
+lib.ttt_status_string.restype = ctypes.c_char_p
+lib.ttt_status_string.argtypes = [_I]
+lib.ttt_abi_version.restype = _I
+lib.ttt_abi_version.argtypes = []
+
+
+def status_string(status: int) -> str:
+    return lib.ttt_status_string(status).decode()
+
+
+def _check(status: int):
+    if status != 0:
+        raise TTTError(status, status_string(status))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TTT_BF16
+    if t.dtype == torch.float32:
+        return TTT_F32
+    raise TypeError(f"Q/K/V must be bf16 or fp32, got {t.dtype}")
+
+
+def _mode_code(mode) -> int:
+    if mode in ("ln", "ln_residual", TTT_LN_RESIDUAL):
+        return TTT_LN_RESIDUAL
+    if mode in ("plain", TTT_PLAIN):
+        return TTT_PLAIN
+    raise ValueError(f"unknown mode {mode!r}")
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return ctypes.c_void_p(handle)
+
+
+class _HostRoundTrip:
+    """Moves CPU inputs to the GPU and device outputs back (end-to-end path)."""
+
+    def __init__(self, tensors):
+        self.on_host = any(t is not None and t.device.type == "cpu" for t in tensors)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if self.on_host else None
+
+    def to_device(self, t):
+        if t is None or not self.on_host:
+            return t
+        if t.device.type != "cpu":
+            return t
+        src = t if t.is_pinned() else t.pin_memory()
+        return src.to(self.device, non_blocking=True)
+
+    def to_host(self, outs):
+        if not self.on_host:
+            return outs
+        host = []
+        for o in outs:
+            if o is None:
+                host.append(None)
+                continue
+            h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+            h.copy_(o, non_blocking=True)
+            host.append(h)
+        torch.cuda.current_stream(self.device).synchronize()
+        return tuple(host)
+
+
+def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *,
+                       mini_batch: int = 16, mode="ln", ln_eps: float = 1e-6, impl: str = "auto",
+                       Z=None, W_T=None, b_T=None, stream=None
+                       ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """TTT-Linear forward scan (see include/ttt.h).  Returns (Z, W_T, b_T)."""
+    rt = _HostRoundTrip([Q, K, V, eta, W0])
+    Q, K, V, eta, W0, b0, ln_gamma, ln_beta = (
+        rt.to_device(x) for x in (Q, K, V, eta, W0, b0, ln_gamma, ln_beta))
+    B, H, T, d = Q.shape
+    m = _mode_code(mode)
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("eta", eta), ("W0", W0), ("b0", b0),
+                    ("ln_gamma", ln_gamma), ("ln_beta", ln_beta)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if K.shape != Q.shape or V.shape != Q.shape or K.dtype != Q.dtype or V.dtype != Q.dtype:
+        raise ValueError("Q, K, V must share shape and dtype")
+    if tuple(eta.shape) != (B, H, T) or tuple(W0.shape) != (B, H, d, d):
+        raise ValueError("eta must be [B,H,T] and W0 [B,H,d,d]")
+    dev = Q.device
+    if Z is None:
+        Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    if W_T is None:
+        W_T = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    if b_T is None and m == TTT_LN_RESIDUAL:
+        b_T = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    st = lib.ttt_linear_forward_impl(
+        B, H, T, d, int(mini_batch), _dtype_code(Q), m, float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
+        _ptr(eta), _ptr(W0), _ptr(b0), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _ptr(W_T),
+        _ptr(b_T), IMPLS[impl], _stream_handle(dev, stream))
+    _check(st)
+    return rt.to_host((Z, W_T, b_T))
+
+
+def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
+                    mini_batch: int = 16, ln_eps: float = 1e-6, Z=None, W1_T=None, b1_T=None,
+                    W2_T=None, b2_T=None, stream=None):
+    """TTT-MLP forward scan (see include/ttt.h).  Returns (Z, W1_T, b1_T, W2_T, b2_T)."""
+    rt = _HostRoundTrip([Q, K, V, eta, W1_0])
+    Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta = (
+        rt.to_device(x) for x in (Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta))
+    B, H, T, d = Q.shape
+    hid = W1_0.shape[-1]
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("eta", eta), ("W1_0", W1_0), ("b1_0", b1_0),
+                    ("W2_0", W2_0), ("b2_0", b2_0), ("ln_gamma", ln_gamma), ("ln_beta", ln_beta)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    dev = Q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    Z = torch.empty((B, H, T, d), **f32) if Z is None else Z
+    W1_T = torch.empty((B, H, d, hid), **f32) if W1_T is None else W1_T
+    b1_T = torch.empty((B, H, hid), **f32) if b1_T is None else b1_T
+    W2_T = torch.empty((B, H, hid, d), **f32) if W2_T is None else W2_T
+    b2_T = torch.empty((B, H, d), **f32) if b2_T is None else b2_T
+    st = lib.ttt_mlp_forward(
+        B, H, T, d, hid, int(mini_batch), _dtype_code(Q), float(ln_eps), _ptr(Q), _ptr(K),
+        _ptr(V), _ptr(eta), _ptr(W1_0), _ptr(b1_0), _ptr(W2_0), _ptr(b2_0), _ptr(ln_gamma),
+        _ptr(ln_beta), _ptr(Z), _ptr(W1_T), _ptr(b1_T), _ptr(W2_T), _ptr(b2_T),
+        _stream_handle(dev, stream))
+    _check(st)
+    return rt.to_host((Z, W1_T, b1_T, W2_T, b2_T))

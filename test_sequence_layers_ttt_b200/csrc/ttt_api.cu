@@ -1,0 +1,176 @@
+// Host layer of the C ABI declared in include/ttt.h: argument validation,
+// kernel-family dispatch and status mapping.  Validation runs entirely on the
+// host and launches nothing when it fails.
+#include <climits>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "ttt_internal.h"
+
+namespace {
+
+using ttt::LinearArgs;
+using ttt::MlpArgs;
+
+struct Span {
+    const void* p;
+    size_t bytes;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(Span a, Span b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+bool check_env() {
+    const char* v = std::getenv("TTT_CHECK");
+    return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+bool valid_mini_batch(int mb) { return mb >= 1 && (mb % 16 == 0 || mb == 1 || mb == 2 || mb == 4 || mb == 8); }
+
+// Outputs must not overlap any other buffer, except that an output state
+// buffer may be exactly its initial-state buffer (in-place update).
+ttt_status check_aliasing(const Span* outs, int n_out, const Span* ins, const int* same_as, int n_in) {
+    for (int o = 0; o < n_out; o++) {
+        for (int i = 0; i < n_in; i++) {
+            if (same_as[o] == i && outs[o].p == ins[i].p) continue;
+            if (overlap(outs[o], ins[i])) return TTT_ERR_ALIAS;
+        }
+        for (int o2 = o + 1; o2 < n_out; o2++)
+            if (overlap(outs[o], outs[o2])) return TTT_ERR_ALIAS;
+    }
+    return TTT_OK;
+}
+
+ttt_status finish(cudaError_t launch, cudaStream_t stream) {
+    if (launch != cudaSuccess) return TTT_ERR_CUDA;
+    if (!check_env()) return TTT_OK;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
+    unsigned int flag = 0;
+    if (ttt::read_and_clear_device_error(&flag) != cudaSuccess) return TTT_ERR_CUDA;
+    return flag ? TTT_ERR_TIMEOUT : TTT_OK;
+}
+
+ttt_status validate_linear(const LinearArgs& a) {
+    if (a.B < 1 || a.H < 1 || a.T < 0 || (long long)a.B * a.H > INT_MAX) return TTT_ERR_SHAPE;
+    if (!valid_mini_batch(a.mini_batch)) return TTT_ERR_SHAPE;
+    if (a.dtype != TTT_BF16 && a.dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (a.mode != TTT_LN_RESIDUAL && a.mode != TTT_PLAIN) return TTT_ERR_UNSUPPORTED;
+    if (a.d != 16 && a.d != 32 && a.d != 64) return TTT_ERR_UNSUPPORTED;
+    const bool ln = a.mode == TTT_LN_RESIDUAL;
+    if (ln && !(a.ln_eps > 0.f)) return TTT_ERR_SHAPE;
+    if (!a.Q || !a.K || !a.V || !a.eta || !a.W0 || !a.Z || !a.W_T) return TTT_ERR_NULL;
+    if (ln && (!a.b0 || !a.gamma || !a.beta || !a.b_T)) return TTT_ERR_NULL;
+    const void* ptrs[] = {a.Q, a.K, a.V, a.eta, a.W0, a.b0, a.gamma, a.beta, a.Z, a.W_T, a.b_T};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TTT_ERR_ALIGN;
+
+    const size_t es = a.dtype == TTT_BF16 ? 2 : 4;
+    const size_t bh = (size_t)a.B * a.H, ntok = bh * (size_t)a.T, d = a.d;
+    Span ins[] = {{a.Q, ntok * d * es},   {a.K, ntok * d * es},      {a.V, ntok * d * es},
+                  {a.eta, ntok * 4},      {a.W0, bh * d * d * 4},    {a.b0, a.b0 ? bh * d * 4 : 0},
+                  {a.gamma, a.gamma ? (size_t)a.H * d * 4 : 0},      {a.beta, a.beta ? (size_t)a.H * d * 4 : 0}};
+    Span outs[] = {{a.Z, ntok * d * 4}, {a.W_T, bh * d * d * 4}, {a.b_T, a.b_T ? bh * d * 4 : 0}};
+    const int same_as[] = {-1, 4, 5};
+    return check_aliasing(outs, 3, ins, same_as, 8);
+}
+
+ttt_status validate_mlp(const MlpArgs& a) {
+    if (a.B < 1 || a.H < 1 || a.T < 0 || (long long)a.B * a.H > INT_MAX) return TTT_ERR_SHAPE;
+    if (!valid_mini_batch(a.mini_batch)) return TTT_ERR_SHAPE;
+    if (a.dtype != TTT_BF16 && a.dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (!ttt::mlp_generic_supports(a)) return TTT_ERR_UNSUPPORTED;
+    if (!(a.ln_eps > 0.f)) return TTT_ERR_SHAPE;
+    const void* req[] = {a.Q, a.K, a.V, a.eta, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma, a.beta,
+                         a.Z, a.W1_T, a.b1_T, a.W2_T, a.b2_T};
+    for (const void* p : req)
+        if (!p) return TTT_ERR_NULL;
+    for (const void* p : req)
+        if (!aligned16(p)) return TTT_ERR_ALIGN;
+    const size_t es = a.dtype == TTT_BF16 ? 2 : 4;
+    const size_t bh = (size_t)a.B * a.H, ntok = bh * (size_t)a.T, d = a.d, hd = a.hidden;
+    Span ins[] = {{a.Q, ntok * d * es},     {a.K, ntok * d * es},   {a.V, ntok * d * es},
+                  {a.eta, ntok * 4},        {a.W1_0, bh * d * hd * 4}, {a.b1_0, bh * hd * 4},
+                  {a.W2_0, bh * hd * d * 4}, {a.b2_0, bh * d * 4},   {a.gamma, (size_t)a.H * d * 4},
+                  {a.beta, (size_t)a.H * d * 4}};
+    Span outs[] = {{a.Z, ntok * d * 4}, {a.W1_T, bh * d * hd * 4}, {a.b1_T, bh * hd * 4},
+                   {a.W2_T, bh * hd * d * 4}, {a.b2_T, bh * d * 4}};
+    const int same_as[] = {-1, 4, 5, 6, 7};
+    return check_aliasing(outs, 5, ins, same_as, 10);
+}
+
+}  // namespace
+
+extern "C" {
+
+ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                                   ttt_mode mode, float ln_eps, const void* Q, const void* K,
+                                   const void* V, const float* eta, const float* W0,
+                                   const float* b0, const float* ln_gamma, const float* ln_beta,
+                                   float* Z, float* W_T, float* b_T, ttt_impl impl,
+                                   ttt_stream_t stream) {
+    LinearArgs a{B, H, T, d, mini_batch, qkv_dtype, mode, ln_eps, Q, K, V, eta,
+                 W0, b0, ln_gamma, ln_beta, Z, W_T, b_T};
+    ttt_status st = validate_linear(a);
+    if (st != TTT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (impl) {
+        case TTT_IMPL_AUTO:
+            if (ttt::linear_tc_supports(a)) return finish(ttt::launch_linear_tc(a, s), s);
+            return finish(ttt::launch_linear_generic(a, s), s);
+        case TTT_IMPL_GENERIC:
+            return finish(ttt::launch_linear_generic(a, s), s);
+        case TTT_IMPL_TENSORCORE:
+            if (!ttt::linear_tc_supports(a)) return TTT_ERR_UNSUPPORTED;
+            return finish(ttt::launch_linear_tc(a, s), s);
+        default:
+            return TTT_ERR_UNSUPPORTED;
+    }
+}
+
+ttt_status ttt_linear_forward(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                              ttt_mode mode, float ln_eps, const void* Q, const void* K,
+                              const void* V, const float* eta, const float* W0, const float* b0,
+                              const float* ln_gamma, const float* ln_beta, float* Z, float* W_T,
+                              float* b_T, ttt_stream_t stream) {
+    return ttt_linear_forward_impl(B, H, T, d, mini_batch, qkv_dtype, mode, ln_eps, Q, K, V, eta,
+                                   W0, b0, ln_gamma, ln_beta, Z, W_T, b_T, TTT_IMPL_AUTO, stream);
+}
+
+ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batch,
+                           ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
+                           const void* V, const float* eta, const float* W1_0, const float* b1_0,
+                           const float* W2_0, const float* b2_0, const float* ln_gamma,
+                           const float* ln_beta, float* Z, float* W1_T, float* b1_T, float* W2_T,
+                           float* b2_T, ttt_stream_t stream) {
+    MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1_0, b1_0,
+              W2_0, b2_0, ln_gamma, ln_beta, Z, W1_T, b1_T, W2_T, b2_T};
+    ttt_status st = validate_mlp(a);
+    if (st != TTT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return finish(ttt::launch_mlp_generic(a, s), s);
+}
+
+const char* ttt_status_string(ttt_status status) {
+    switch (status) {
+        case TTT_OK: return "TTT_OK";
+        case TTT_ERR_NULL: return "TTT_ERR_NULL: a required pointer is NULL";
+        case TTT_ERR_SHAPE: return "TTT_ERR_SHAPE: B, H, T, mini_batch or ln_eps out of range";
+        case TTT_ERR_DTYPE: return "TTT_ERR_DTYPE: unknown element type";
+        case TTT_ERR_ALIGN: return "TTT_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case TTT_ERR_ALIAS: return "TTT_ERR_ALIAS: an output overlaps another buffer";
+        case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED: shape, mode or kernel family not built";
+        case TTT_ERR_CUDA: return "TTT_ERR_CUDA: CUDA launch or execution error";
+        case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+        default: return "TTT_ERR_UNKNOWN";
+    }
+}
+
+int ttt_abi_version(void) { return 100; }
+
+}  // extern "C"

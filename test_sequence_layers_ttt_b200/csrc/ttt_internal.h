@@ -1,0 +1,41 @@
+// Internal launch interface between the host layer (ttt_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/ttt.h"
+
+namespace ttt {
+
+struct LinearArgs {
+    int B, H, T, d, mini_batch;
+    ttt_dtype dtype;
+    ttt_mode mode;
+    float ln_eps;
+    const void *Q, *K, *V;
+    const float *eta, *W0, *b0, *gamma, *beta;
+    float *Z, *W_T, *b_T;
+};
+
+struct MlpArgs {
+    int B, H, T, d, hidden, mini_batch;
+    ttt_dtype dtype;
+    float ln_eps;
+    const void *Q, *K, *V;
+    const float *eta, *W1_0, *b1_0, *W2_0, *b2_0, *gamma, *beta;
+    float *Z, *W1_T, *b1_T, *W2_T, *b2_T;
+};
+
+bool linear_generic_supports(const LinearArgs& a);
+cudaError_t launch_linear_generic(const LinearArgs& a, cudaStream_t stream);
+
+bool linear_tc_supports(const LinearArgs& a);
+cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream);
+
+bool mlp_generic_supports(const MlpArgs& a);
+cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);
+
+// Device-side error word set by kernels that abandon a bounded wait.
+cudaError_t read_and_clear_device_error(unsigned int* out);
+
+}  // namespace ttt

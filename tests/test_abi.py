@@ -1,0 +1,138 @@
+"""The C-ABI library loads, exports every symbol include/ttt.h declares, and
+rejects bad arguments on the host with the documented status codes.
+
+Every call here carries at least one argument error, so validation returns
+before anything is launched; the pointer values are never dereferenced.
+No GPU is needed.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttt.h")
+
+b = pytest.importorskip("test_sequence_layers_ttt_b200._binding")
+
+OK, NULL, SHAPE, DTYPE, ALIGN, ALIAS, UNSUP = 0, 1, 2, 3, 4, 5, 6
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:ttt_status|const char\*|int)\s+(ttt_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_status_string",
+              "ttt_linear_forward_impl", "ttt_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(b.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ttt.h but not exported"
+
+
+def test_status_strings():
+    for code, name in enumerate(b.STATUS):
+        assert b.status_string(code).startswith(name)
+    assert b.status_string(99) == "TTT_ERR_UNKNOWN"
+    assert b.lib.ttt_abi_version() == 100
+
+
+# Fake, 16-byte aligned, non-overlapping device addresses.  Never dereferenced:
+# every case below fails validation first.
+BASE = 1 << 40
+STRIDE = 1 << 34
+
+
+def fake(i):
+    return BASE + i * STRIDE
+
+
+def linear_call(B=1, H=2, T=64, d=64, mb=16, dtype=0, mode=0, eps=1e-6, ptrs=None, impl=0):
+    p = [fake(i) for i in range(11)] if ptrs is None else ptrs
+    return b.lib.ttt_linear_forward_impl(B, H, T, d, mb, dtype, mode, eps, *p, impl, None)
+
+
+def mlp_call(B=1, H=2, T=64, d=64, hid=256, mb=16, dtype=0, eps=1e-6, ptrs=None):
+    p = [fake(i) for i in range(15)] if ptrs is None else ptrs
+    return b.lib.ttt_mlp_forward(B, H, T, d, hid, mb, dtype, eps, *p, None)
+
+
+def with_ptr(i, value, n=11):
+    p = [fake(k) for k in range(n)]
+    p[i] = value
+    return p
+
+
+# argument order: Q K V eta W0 b0 gamma beta Z W_T b_T
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4, 8, 9])
+def test_linear_null_required_pointer(idx):
+    assert linear_call(ptrs=with_ptr(idx, None)) == NULL
+
+
+@pytest.mark.parametrize("idx", [5, 6, 7, 10])
+def test_linear_ln_mode_needs_bias_and_ln_params(idx):
+    assert linear_call(ptrs=with_ptr(idx, None)) == NULL
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), SHAPE), (dict(H=0), SHAPE), (dict(T=-1), SHAPE), (dict(mb=0), SHAPE),
+    (dict(mb=12), SHAPE), (dict(mb=24), SHAPE), (dict(mb=3), SHAPE),
+    (dict(eps=0.0), SHAPE), (dict(eps=-1.0), SHAPE),
+    (dict(dtype=7), DTYPE), (dict(d=48), UNSUP), (dict(d=128), UNSUP), (dict(mode=5), UNSUP),
+    (dict(B=1 << 16, H=1 << 16), SHAPE),
+])
+def test_linear_bad_shapes(kw, code):
+    assert linear_call(**kw) == code
+
+
+@pytest.mark.parametrize("idx", range(11))
+def test_linear_misaligned_pointer(idx):
+    assert linear_call(ptrs=with_ptr(idx, fake(idx) + 8)) == ALIGN
+
+
+def test_linear_z_overlapping_q_is_alias():
+    p = [fake(k) for k in range(11)]
+    p[8] = p[0] + 256  # Z inside Q
+    assert linear_call(ptrs=p) == ALIAS
+
+
+def test_linear_partial_state_overlap_is_alias():
+    p = [fake(k) for k in range(11)]
+    p[9] = p[4] + 16  # W_T overlaps W0 but is not the same pointer
+    assert linear_call(ptrs=p) == ALIAS
+
+
+def test_linear_outputs_overlapping_each_other_is_alias():
+    p = [fake(k) for k in range(11)]
+    p[10] = p[8] + 64  # b_T inside Z
+    assert linear_call(ptrs=p) == ALIAS
+
+
+# MLP: Q K V eta W1 b1 W2 b2 gamma beta Z W1_T b1_T W2_T b2_T
+@pytest.mark.parametrize("idx", range(15))
+def test_mlp_null_pointer(idx):
+    assert mlp_call(ptrs=with_ptr(idx, None, 15)) == NULL
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=32), UNSUP), (dict(hid=128), UNSUP), (dict(mb=10), SHAPE), (dict(B=0), SHAPE),
+    (dict(dtype=3), DTYPE), (dict(eps=0.0), SHAPE)])
+def test_mlp_bad_shapes(kw, code):
+    assert mlp_call(**kw) == code
+
+
+def test_mlp_alias_and_align():
+    p = [fake(k) for k in range(15)]
+    p[10] = p[2] + 1024  # Z inside V
+    assert mlp_call(ptrs=p) == ALIAS
+    assert mlp_call(ptrs=with_ptr(13, fake(13) + 4, 15)) == ALIGN

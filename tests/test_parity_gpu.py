@@ -1,0 +1,247 @@
+"""Parity of the CUDA library (through the C ABI) against the float64 oracle.
+
+Bar (stated for the TTT forward scan): max |GPU - oracle| <= 1e-4 * RMS(Z)
+with fp32 Q/K/V and <= 3e-3 * RMS(Z) with bf16 Q/K/V and fp32 state.  The
+final state is held to the same factor times its own RMS.  Both sides consume
+identical input bits from the seeded generators.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from test_sequence_layers_ttt_b200.inputs import (MODE_PLAIN, WORKLOADS, make_inputs,
+                                                  select_heads)
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 3e-3}
+LINEAR_KEYS = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+MLP_KEYS = ("Q", "K", "V", "eta", "W1_0", "b1_0", "W2_0", "b2_0", "gamma", "beta")
+
+
+@pytest.fixture(scope="module")
+def ttt(cuda_device):
+    from test_sequence_layers_ttt_b200 import _binding
+    return _binding
+
+
+def to_cuda(inp):
+    return {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+
+
+def rms(x):
+    return float(np.sqrt(np.mean(np.square(x, dtype=np.float64))))
+
+
+def assert_close(got, ref, factor, what, denom=None):
+    got = np.asarray(got, dtype=np.float64)
+    d = rms(ref) if denom is None else denom
+    err = float(np.abs(got - ref).max()) if got.size else 0.0
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert err <= factor * d, f"{what}: max err {err:.3e} > {factor:g} * RMS {d:.3e}"
+    return err / d if d else 0.0
+
+
+def gpu_linear(ttt, w, inp, impl="auto", mini_batch=None):
+    g = to_cuda(inp)
+    plain = w.mode == MODE_PLAIN
+    Z, W_T, b_T = ttt.ttt_linear_forward(
+        g["Q"], g["K"], g["V"], g["eta"], g["W0"], None if plain else g["b0"],
+        None if plain else g["gamma"], None if plain else g["beta"],
+        mini_batch=mini_batch or w.mini_batch, mode="plain" if plain else "ln",
+        ln_eps=w.ln_eps, impl=impl)
+    torch.cuda.synchronize()
+    return Z.cpu().numpy(), W_T.cpu().numpy(), None if b_T is None else b_T.cpu().numpy()
+
+
+def oracle_linear(w, inp, mini_batch=None):
+    return oracle.ttt_linear(*(inp[k] for k in LINEAR_KEYS), mini_batch or w.mini_batch, w.mode,
+                             w.ln_eps)
+
+
+def compare_linear(ttt, w, inp, impl="auto", mini_batch=None):
+    Z, W_T, b_T = gpu_linear(ttt, w, inp, impl, mini_batch)
+    Zo, Wo, bo = oracle_linear(w, inp, mini_batch)
+    f = TOL[w.dtype]
+    e = assert_close(Z, Zo, f, "Z")
+    assert_close(W_T, Wo, f, "W_T")
+    if b_T is not None and np.any(bo):
+        assert_close(b_T, bo, f, "b_T", denom=max(rms(bo), rms(Wo)))
+    return e
+
+
+# ---------------------------------------------------------------- TTT-Linear
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("impl", ["auto", "generic"])
+def test_linear_tiny_f32(ttt, seed, impl):
+    w = WORKLOADS["linear_tiny_f32"]
+    compare_linear(ttt, w, make_inputs(w, seed), impl)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_theorem1_f32(ttt, seed):
+    """Theorem-1 workload, full size: also equals causal linear attention."""
+    w = WORKLOADS["theorem1_f32"]
+    inp = make_inputs(w, seed)
+    compare_linear(ttt, w, inp)
+    Z, _, _ = gpu_linear(ttt, w, inp)
+    Q, K, V = (inp[k].double() for k in "QKV")
+    Zref = (torch.tril(Q @ K.transpose(-1, -2)) @ V).numpy()
+    assert_close(Z, Zref, TOL["f32"], "Z vs linear attention")
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("name,shape", [
+    ("linear_125m_2k", dict(B=2, H=3, T=200)),       # several chunks + ragged tail (200 = 12*16 + 8)
+    ("linear_1p3b_32k", dict(B=1, H=4, T=1000)),
+])
+@pytest.mark.parametrize("impl", ["auto", "generic"])
+def test_linear_bf16_reduced(ttt, seed, name, shape, impl):
+    w = WORKLOADS[name].with_shape(**shape)
+    compare_linear(ttt, w, make_inputs(w, seed), impl)
+
+
+def test_linear_125m_full(ttt):
+    w = WORKLOADS["linear_125m_2k"]
+    compare_linear(ttt, w, make_inputs(w, 0))
+
+
+def test_linear_1p3b_32k_full_sampled_heads(ttt):
+    """The benchmarked launch: all 64 scans of 32k tokens on the GPU, four of
+    them checked end to end against the oracle."""
+    w = WORKLOADS["linear_1p3b_32k"]
+    inp = make_inputs(w, 0)
+    Z, W_T, b_T = gpu_linear(ttt, w, inp)
+    pairs = [(0, 0), (0, 17), (1, 5), (1, 31)]
+    sel = select_heads(inp, pairs)
+    Zo, Wo, bo = oracle_linear(w, sel)
+    f = TOL["bf16"]
+    for i, (bb, hh) in enumerate(pairs):
+        assert_close(Z[bb, hh], Zo[0, i], f, f"Z[{bb},{hh}]", denom=rms(Zo))
+        assert_close(W_T[bb, hh], Wo[0, i], f, f"W_T[{bb},{hh}]", denom=rms(Wo))
+    assert np.isfinite(Z).all()
+
+
+@pytest.mark.parametrize("mb", [1, 2, 4, 8, 32, 64])
+def test_linear_mini_batch_sizes(ttt, mb):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=192)
+    compare_linear(ttt, w, make_inputs(w, 3), mini_batch=mb)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_linear_dims_dtypes_modes(ttt, d, dtype, mode):
+    w = WORKLOADS["linear_tiny_f32"].with_shape(B=2, H=2, T=72, d=d, dtype=dtype, mode=mode)
+    compare_linear(ttt, w, make_inputs(w, 4))
+
+
+@pytest.mark.parametrize("T", [0, 1, 15, 17])
+def test_linear_short_and_empty_sequences(ttt, T):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=T)
+    inp = make_inputs(w, 5)
+    Z, W_T, b_T = gpu_linear(ttt, w, inp)
+    if T == 0:
+        np.testing.assert_array_equal(W_T, inp["W0"].numpy())
+        np.testing.assert_array_equal(b_T, inp["b0"].numpy())
+        assert Z.size == 0
+    else:
+        compare_linear(ttt, w, inp)
+
+
+def test_linear_in_place_state_and_continuation(ttt):
+    """W_T may be W0 (in-place).  Splitting the sequence at a mini-batch
+    boundary and feeding the state back gives the identical result."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=2, T=256)
+    g = to_cuda(make_inputs(w, 6))
+    args = lambda sl: [g[k][:, :, sl].contiguous() for k in ("Q", "K", "V", "eta")]
+    Zf, Wf, bf = ttt.ttt_linear_forward(*args(slice(None)), g["W0"], g["b0"], g["gamma"], g["beta"])
+    W, b = g["W0"].clone(), g["b0"].clone()
+    Za, _, _ = ttt.ttt_linear_forward(*args(slice(0, 128)), W, b, g["gamma"], g["beta"], W_T=W, b_T=b)
+    Zb, _, _ = ttt.ttt_linear_forward(*args(slice(128, None)), W, b, g["gamma"], g["beta"], W_T=W, b_T=b)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([Za, Zb], dim=2), Zf)
+    assert torch.equal(W, Wf) and torch.equal(b, bf)
+
+
+@pytest.mark.parametrize("impl", ["auto", "generic"])
+def test_linear_deterministic(ttt, impl):
+    w = WORKLOADS["linear_1p3b_32k"].with_shape(B=2, H=4, T=512)
+    g = to_cuda(make_inputs(w, 7))
+    a = ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl=impl)
+    b = ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl=impl)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+def test_linear_tensorcore_refuses_other_shapes(ttt):
+    w = WORKLOADS["linear_tiny_f32"]
+    g = to_cuda(make_inputs(w, 0))
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl="tensorcore")
+    assert ei.value.status == 6
+
+
+def test_linear_host_buffers_end_to_end(ttt):
+    """CPU tensors in, CPU tensors out: the same numbers as the device path."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=3, T=96)
+    inp = make_inputs(w, 8)
+    Zh, Wh, bh = ttt.ttt_linear_forward(*(inp[k] for k in LINEAR_KEYS))
+    assert Zh.device.type == "cpu"
+    Zd, Wd, bd = gpu_linear(ttt, w, inp)
+    np.testing.assert_array_equal(Zh.numpy(), Zd)
+    np.testing.assert_array_equal(Wh.numpy(), Wd)
+
+
+# ------------------------------------------------------------------ TTT-MLP
+
+def gpu_mlp(ttt, w, inp, mini_batch=None):
+    g = to_cuda(inp)
+    out = ttt.ttt_mlp_forward(*(g[k] for k in MLP_KEYS), mini_batch=mini_batch or w.mini_batch,
+                              ln_eps=w.ln_eps)
+    torch.cuda.synchronize()
+    return [o.cpu().numpy() for o in out]
+
+
+def oracle_mlp(w, inp, mini_batch=None):
+    return oracle.ttt_mlp(*(inp[k] for k in MLP_KEYS), mini_batch or w.mini_batch, w.ln_eps)
+
+
+def compare_mlp(ttt, w, inp, mini_batch=None, pairs=None):
+    out = gpu_mlp(ttt, w, inp, mini_batch)
+    if pairs is not None:
+        ref = oracle_mlp(w, select_heads(inp, pairs), mini_batch)
+        out = [np.stack([o[bb, hh] for bb, hh in pairs])[None] for o in out]
+    else:
+        ref = oracle_mlp(w, inp, mini_batch)
+    f = TOL[w.dtype]
+    assert_close(out[0], ref[0], f, "Z")
+    for name, o, r in zip(("W1_T", "b1_T", "W2_T", "b2_T"), out[1:], ref[1:]):
+        scale = rms(r) if np.any(r) else 1.0
+        assert_close(o, r, f, name, denom=max(scale, 1e-3 * rms(ref[1])))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_mlp_reduced(ttt, seed):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=200)
+    compare_mlp(ttt, w, make_inputs(w, seed))
+
+
+@pytest.mark.parametrize("mb", [1, 8, 32])
+def test_mlp_mini_batch_sizes(ttt, mb):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=96)
+    compare_mlp(ttt, w, make_inputs(w, 3), mini_batch=mb)
+
+
+def test_mlp_f32_inputs(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=64, dtype="f32")
+    compare_mlp(ttt, w, make_inputs(w, 2))
+
+
+def test_mlp_full_sampled_heads(ttt):
+    w = WORKLOADS["mlp_8k"]
+    compare_mlp(ttt, w, make_inputs(w, 0), pairs=[(0, 0), (2, 7), (3, 11)])
