@@ -294,7 +294,9 @@ def run_ours(args, world, rank, local):
         hbm, peak_kind = load_peaks()
         ab = algorithmic_bytes(w)
         achieved = ab / (kernel_ms * 1e-3) / 1e9
-        kname = "ttt_linear_tc_kernel" if args.kernel != "generic" else "ttt_linear_generic_kernel"
+        family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
+            w.B, w.H, w.T, w.d, w.mini_batch, w.dtype, w.mode)
+        kname = {"tensorcore": "ttt_linear_tc_kernel", "generic": "ttt_linear_generic_kernel"}[family]
         traffic = recorded_traffic(kname, w.name)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -310,7 +312,7 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
-            "kernel_impl": args.kernel,
+            "kernel_impl": family,
             "tflops_achieved": algorithmic_flops(w) / (kernel_ms * 1e-3) / 1e12,
         }
         print(json.dumps(line), flush=True)

@@ -45,8 +45,9 @@
  *   Aliasing    W_T may be the same pointer as W0 (and b_T as b0) for an
  *               in-place state update; any other overlap between an output
  *               (Z, W_T, b_T) and any other buffer is TTT_ERR_ALIAS.
- *   Shapes      B, H >= 1; T >= 0 (T = 0 copies the state); mini_batch >= 1
- *               and either a multiple of 16 or one of 1, 2, 4, 8.
+ *   Shapes      B, H >= 1; T >= 0; mini_batch >= 1 and either a multiple of
+ *               16 or one of 1, 2, 4, 8.  T = 0 copies the state; the token
+ *               buffers (Q, K, V, eta, Z) are then empty and may be NULL.
  *   Stream      Work is enqueued on `stream` (0 = legacy default stream); the
  *               call does not synchronise.
  *   Errors      Argument errors are detected on the host before anything is
@@ -121,6 +122,11 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch,
                                    const float* eta, const float* W0, const float* b0,
                                    const float* ln_gamma, const float* ln_beta, float* Z,
                                    float* W_T, float* b_T, ttt_impl impl, ttt_stream_t stream);
+
+/* Kernel family TTT_IMPL_AUTO would run for these arguments (TTT_IMPL_AUTO if
+ * no family covers them).  Pure host query; launches nothing. */
+ttt_impl ttt_linear_pick_impl(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                              ttt_mode mode);
 
 /*
  * TTT-MLP forward scan, f(x) = x + LN(GELU(x W1 + b1) W2 + b2).

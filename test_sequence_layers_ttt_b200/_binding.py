@@ -50,6 +50,16 @@ lib.ttt_status_string.restype = ctypes.c_char_p
 lib.ttt_status_string.argtypes = [_I]
 lib.ttt_abi_version.restype = _I
 lib.ttt_abi_version.argtypes = []
+lib.ttt_linear_pick_impl.restype = _I
+lib.ttt_linear_pick_impl.argtypes = [_I] * 7
+
+
+def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
+    """Kernel family the library's AUTO dispatch runs for these arguments."""
+    code = lib.ttt_linear_pick_impl(B, H, T, d, mini_batch,
+                                    TTT_BF16 if qkv_dtype in ("bf16", torch.bfloat16) else TTT_F32,
+                                    _mode_code(mode))
+    return {0: "none", 1: "generic", 2: "tensorcore"}[code]
 
 
 def status_string(status: int) -> str:

@@ -64,7 +64,9 @@ ttt_status validate_linear(const LinearArgs& a) {
     if (a.d != 16 && a.d != 32 && a.d != 64) return TTT_ERR_UNSUPPORTED;
     const bool ln = a.mode == TTT_LN_RESIDUAL;
     if (ln && !(a.ln_eps > 0.f)) return TTT_ERR_SHAPE;
-    if (!a.Q || !a.K || !a.V || !a.eta || !a.W0 || !a.Z || !a.W_T) return TTT_ERR_NULL;
+    // with T == 0 the token buffers are empty and may be NULL
+    if (a.T > 0 && (!a.Q || !a.K || !a.V || !a.eta || !a.Z)) return TTT_ERR_NULL;
+    if (!a.W0 || !a.W_T) return TTT_ERR_NULL;
     if (ln && (!a.b0 || !a.gamma || !a.beta || !a.b_T)) return TTT_ERR_NULL;
     const void* ptrs[] = {a.Q, a.K, a.V, a.eta, a.W0, a.b0, a.gamma, a.beta, a.Z, a.W_T, a.b_T};
     for (const void* p : ptrs)
@@ -86,12 +88,13 @@ ttt_status validate_mlp(const MlpArgs& a) {
     if (a.dtype != TTT_BF16 && a.dtype != TTT_F32) return TTT_ERR_DTYPE;
     if (!ttt::mlp_generic_supports(a)) return TTT_ERR_UNSUPPORTED;
     if (!(a.ln_eps > 0.f)) return TTT_ERR_SHAPE;
-    const void* req[] = {a.Q, a.K, a.V, a.eta, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma, a.beta,
-                         a.Z, a.W1_T, a.b1_T, a.W2_T, a.b2_T};
+    const void* req[] = {a.Q, a.K, a.V, a.eta, a.Z, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma,
+                         a.beta, a.W1_T, a.b1_T, a.W2_T, a.b2_T};
+    // with T == 0 the token buffers (the first five) are empty and may be NULL
+    for (int i = a.T > 0 ? 0 : 5; i < 15; i++)
+        if (!req[i]) return TTT_ERR_NULL;
     for (const void* p : req)
-        if (!p) return TTT_ERR_NULL;
-    for (const void* p : req)
-        if (!aligned16(p)) return TTT_ERR_ALIGN;
+        if (p && !aligned16(p)) return TTT_ERR_ALIGN;
     const size_t es = a.dtype == TTT_BF16 ? 2 : 4;
     const size_t bh = (size_t)a.B * a.H, ntok = bh * (size_t)a.T, d = a.d, hd = a.hidden;
     Span ins[] = {{a.Q, ntok * d * es},     {a.K, ntok * d * es},   {a.V, ntok * d * es},
@@ -131,6 +134,14 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, t
         default:
             return TTT_ERR_UNSUPPORTED;
     }
+}
+
+ttt_impl ttt_linear_pick_impl(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                              ttt_mode mode) {
+    LinearArgs a{B, H, T, d, mini_batch, qkv_dtype, mode, 1e-6f, nullptr, nullptr, nullptr,
+                 nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    if (ttt::linear_tc_supports(a)) return TTT_IMPL_TENSORCORE;
+    return ttt::linear_generic_supports(a) ? TTT_IMPL_GENERIC : TTT_IMPL_AUTO;
 }
 
 ttt_status ttt_linear_forward(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,

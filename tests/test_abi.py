@@ -24,13 +24,14 @@ OK, NULL, SHAPE, DTYPE, ALIGN, ALIAS, UNSUP = 0, 1, 2, 3, 4, 5, 6
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:ttt_status|const char\*|int)\s+(ttt_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:ttt_status|ttt_impl|const char\*|int)\s+(ttt_\w+)\s*\(",
+                                 text, re.M)))
 
 
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_status_string",
-              "ttt_linear_forward_impl", "ttt_abi_version"):
+              "ttt_linear_forward_impl", "ttt_abi_version", "ttt_linear_pick_impl"):
         assert n in names
 
 
@@ -136,3 +137,18 @@ def test_mlp_alias_and_align():
     p[10] = p[2] + 1024  # Z inside V
     assert mlp_call(ptrs=p) == ALIAS
     assert mlp_call(ptrs=with_ptr(13, fake(13) + 4, 15)) == ALIGN
+
+
+def test_pick_impl_is_a_host_query():
+    f = b.lib.ttt_linear_pick_impl
+    assert f(1, 2, 64, 16, 16, 1, 0) == 1        # fp32 d=16: generic
+    assert f(1, 2, 64, 48, 16, 0, 0) == 0        # d=48: nothing
+    assert f(2, 32, 32768, 64, 16, 0, 0) in (1, 2)
+
+
+def test_empty_sequence_allows_null_token_buffers_but_not_state():
+    p = [fake(k) for k in range(11)]
+    for i in (0, 1, 2, 3, 8):
+        p[i] = None
+    p[4] = None  # W0 is still required
+    assert linear_call(T=0, ptrs=p) == NULL
