@@ -59,7 +59,10 @@
  *               bounded wait (its outputs are then undefined).
  *   Threads     Entry points are re-entrant.
  *   Continuation  Feeding W_T (b_T) back as W0 (b0) continues the sequence
- *               exactly when the split falls on a mini-batch boundary.
+ *               when the split falls on a mini-batch boundary (bit for bit in
+ *               the generic family; the tensor-core family reaches the first
+ *               chunk after a split by an algebraically equal route, so the
+ *               results agree up to rounding).
  */
 #ifndef TTT_B200_TTT_H
 #define TTT_B200_TTT_H
