@@ -71,10 +71,13 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
 }
 
 // ---------------------------------------------------------------- mma.sync
-// D = A * B + D, m16n8k16, bf16 operands, fp32 accumulate.
+// D = A * B + D, m16n8k16, bf16 operands, fp32 accumulate.  A pure function of
+// its register operands (not volatile), so the compiler may interleave
+// independent products; back-to-back products on one accumulator wait for the
+// previous result.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

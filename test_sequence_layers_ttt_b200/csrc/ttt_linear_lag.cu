@@ -119,7 +119,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                       const float* __restrict__ gamma, const float* __restrict__ beta,
                       float* __restrict__ Z, float* W_T, float* b_T, int drop_chunk) {
     extern __shared__ unsigned char smem_raw[];
-    LagSmem& s = *reinterpret_cast<LagSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte alignment (128-byte TMA swizzle) by offsetting the shared array itself, so every
+    // access through `s` stays a shared-memory access (an integer round trip would make them generic)
+    LagSmem& s = *reinterpret_cast<LagSmem*>(smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int bh = blockIdx.x, h = bh % H;
