@@ -10,6 +10,8 @@ Multi-GPU (torchrun): every rank runs its own instance of the workload (the
 (batch, head) scans are independent; no collective on the data path), so
 scaling is weak and value = all ranks' tokens / max-over-ranks time.
 
+--workload selects another of the synthetic workloads (the 125M-layer shape,
+or the TTT-MLP layer, which reports against the bf16 tensor-core peak).
 --impl reference times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only).
 """
@@ -33,8 +35,17 @@ sys.path.insert(0, ROOT)
 from test_sequence_layers_ttt_b200.inputs import WORKLOADS, make_inputs, select_heads  # noqa: E402
 
 METRIC = "TTT forward tokens/sec on 1 B200 (1.3B-layer shape, 32k ctx); % of roofline"
+
+
+def metric_name(w) -> str:
+    if w.name == "linear_1p3b_32k":
+        return METRIC
+    shape = {"linear_125m_2k": "125M-layer shape, 2k ctx", "mlp_8k": "TTT-MLP layer, 8k ctx"}[w.name]
+    return f"TTT forward tokens/sec on 1 B200 ({shape}); % of roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 KEYS = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+KEYS_MLP = ("Q", "K", "V", "eta", "W1_0", "b1_0", "W2_0", "b2_0", "gamma", "beta")
 
 
 def algorithmic_bytes(w) -> int:
@@ -42,22 +53,30 @@ def algorithmic_bytes(w) -> int:
     once and written once per (batch, head), gamma/beta once."""
     es = 2 if w.dtype == "bf16" else 4
     per_tok = 3 * w.d * es + 4 + 4 * w.d
-    state = 2 * (w.d * w.d + w.d) * 4
+    if w.kind == "mlp":
+        state = 2 * (2 * w.d * w.hidden + w.hidden + w.d) * 4
+    else:
+        state = 2 * (w.d * w.d + w.d) * 4
     return w.head_tokens * per_tok + w.B * w.H * state + 2 * w.H * w.d * 4
 
 
 def algorithmic_flops(w) -> int:
-    """6 d^2 (X W, Q W, update) + 4*16*d (Q X^T, A G) per head-token."""
+    """Per head-token.  Linear: 6 d^2 (X W, Q W, update) + 4*16*d (Q X^T, A G).
+    MLP (hidden h): 7 products of 2 d h (two layers on K, two on Q, the hidden
+    gradient, two updates) + 2*16*(2d + 2h) (the causal 16x16 terms)."""
+    if w.kind == "mlp":
+        return w.head_tokens * (7 * 2 * w.d * w.hidden + 2 * 16 * (2 * w.d + 2 * w.hidden))
     return w.head_tokens * (6 * w.d * w.d + 4 * 16 * w.d)
 
 
 def load_peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s burst, 'measured' | 'fallback')."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as fh:
             p = json.load(fh)
-        return float(p["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash() -> str:
@@ -70,17 +89,18 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel sources changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+    the committed ncu summary, or None when the kernel sources changed since the
+    counters were taken.  Lines: kernel workload source_hash bytes."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
-        rec = json.load(fh)
-    entry = rec.get(f"{kernel}:{workload}")
-    if not entry or entry.get("source_hash") != kernel_source_hash():
-        return None
-    return entry.get("dram_bytes_per_launch")
+        for line in fh:
+            f = line.split()
+            if len(f) == 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
+                return int(f[3]) if f[2] == kernel_source_hash() else None
+    return None
 
 
 class ClockSampler:
@@ -177,15 +197,21 @@ def cpu_oracle_sample(w, inp, target_s: float):
     B, H = inp["Q"].shape[:2]
     pairs_all = [(b, h) for b in range(B) for h in range(H)]
     # calibrate on one scan
+    def run(sel, threads):
+        if w.kind == "mlp":
+            oracle.ttt_mlp(*(sel[k] for k in KEYS_MLP), w.mini_batch, w.ln_eps, threads=threads)
+        else:
+            oracle.ttt_linear(*(sel[k] for k in KEYS), w.mini_batch, w.mode, w.ln_eps, threads=threads)
+
     sel = select_heads(inp, pairs_all[:1])
     t0 = time.perf_counter()
-    oracle.ttt_linear(*(sel[k] for k in KEYS), w.mini_batch, w.mode, w.ln_eps, threads=1)
+    run(sel, 1)
     one = time.perf_counter() - t0
     n = max(1, min(len(pairs_all), int(target_s / max(one, 1e-6) * min(cores, len(pairs_all)))))
     n = max(min(n, len(pairs_all)), 1)
     sel = select_heads(inp, pairs_all[:n])
     t0 = time.perf_counter()
-    oracle.ttt_linear(*(sel[k] for k in KEYS), w.mini_batch, w.mode, w.ln_eps, threads=cores)
+    run(sel, cores)
     dt = time.perf_counter() - t0
     tokens = n * w.T / w.H
     used = min(cores, n)
@@ -203,14 +229,15 @@ def run_reference(args, world, rank):
         cpu_oracle_sample(w, inp, 0.5)
     vals, samples = [], None
     t_start = time.perf_counter()
+    per_step = min(args.ref_seconds, 150.0 / max(args.steps, 1))  # whole run within a few minutes
     for _ in range(args.steps):
-        r = cpu_oracle_sample(w, inp, args.ref_seconds)
+        r = cpu_oracle_sample(w, inp, per_step)
         vals.append(r["value"])
         samples = r
     elapsed = time.perf_counter() - t_start
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": metric_name(w), "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -225,7 +252,9 @@ def run_reference(args, world, rank):
 
 def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "mini_batch": w.mini_batch,
-            "qkv_dtype": w.dtype, "state_dtype": "f32", "inner_model": "x + LN(xW + b)",
+            "qkv_dtype": w.dtype, "state_dtype": "f32",
+            "inner_model": (f"x + LN(MLP {w.d}->{w.hidden}->{w.d}, GELU)" if w.kind == "mlp"
+                            else "x + LN(xW + b)"),
             "l2": "inputs (Q/K/V/eta) larger than the 126 MB L2; no flush"}
 
 
@@ -237,13 +266,31 @@ def run_ours(args, world, rank, local):
     host = make_inputs(w, args.seed + rank)
     g = {k: v.to(dev) for k, v in host.items()}
     Z = torch.empty((w.B, w.H, w.T, w.d), dtype=torch.float32, device=dev)
-    W_T = torch.empty_like(g["W0"])
-    b_T = torch.empty_like(g["b0"])
     stream = torch.cuda.current_stream(dev)
+    if w.kind == "mlp":
+        keys = KEYS_MLP
+        state = {n: torch.empty_like(g[n + "_0"]) for n in ("W1", "b1", "W2", "b2")}
+        outs = [Z, *state.values()]
 
-    def step():
-        ttt.ttt_linear_forward(*(g[k] for k in KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps,
-                               impl=args.kernel, Z=Z, W_T=W_T, b_T=b_T, stream=stream)
+        def call(inputs, **kw):
+            return ttt.ttt_mlp_forward(*(inputs[k] for k in keys), mini_batch=w.mini_batch,
+                                       ln_eps=w.ln_eps, **kw)
+
+        def step():
+            call(g, Z=Z, W1_T=state["W1"], b1_T=state["b1"], W2_T=state["W2"], b2_T=state["b2"],
+                 stream=stream)
+    else:
+        keys = KEYS
+        W_T = torch.empty_like(g["W0"])
+        b_T = torch.empty_like(g["b0"])
+        outs = [Z, W_T, b_T]
+
+        def call(inputs, **kw):
+            return ttt.ttt_linear_forward(*(inputs[k] for k in keys), mini_batch=w.mini_batch,
+                                          ln_eps=w.ln_eps, **kw)
+
+        def step():
+            call(g, impl=args.kernel, Z=Z, W_T=W_T, b_T=b_T, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -272,17 +319,16 @@ def run_ours(args, world, rank, local):
     value = tokens_per_step / (ms_per_step * 1e-3)
 
     # end to end through the public API with pinned host buffers
-    host_in = {k: v.pin_memory() for k, v in host.items()}
+    host_in = {k: v.pin_memory() for k, v in host.items() if v is not None}
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = (Z.numel() + W_T.numel() + b_T.numel()) * 4
-    ttt.ttt_linear_forward(*(host_in[k] for k in KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    call(host_in)
     torch.cuda.synchronize(dev)
     dist_barrier(world)
     e2e_steps = max(1, min(args.steps, 3))
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
-        ttt.ttt_linear_forward(*(host_in[k] for k in KEYS), mini_batch=w.mini_batch,
-                               ln_eps=w.ln_eps)  # returns after the device->host copies finish
+        call(host_in)  # returns after the device->host copies finish
     e2e_s = dist_max((time.perf_counter() - t0) / e2e_steps, world)
     e2e_value = tokens_per_step / e2e_s
 
@@ -291,29 +337,35 @@ def run_ours(args, world, rank, local):
         cpu_base = cpu_oracle_sample(w, host, args.ref_seconds)
 
     if rank == 0:
-        hbm, peak_kind = load_peaks()
+        hbm, bf16_tf, peak_kind = load_peaks()
         ab = algorithmic_bytes(w)
-        achieved = ab / (kernel_ms * 1e-3) / 1e9
-        family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
-            w.B, w.H, w.T, w.d, w.mini_batch, w.dtype, w.mode)
-        kname = {"tensorcore": "ttt_linear_tc_kernel", "generic": "ttt_linear_generic_kernel"}[family]
+        af = algorithmic_flops(w)
+        if w.kind == "mlp":
+            family, kname = "generic", "ttt_mlp_generic_kernel"
+            achieved, peak, bound, unit = af / (kernel_ms * 1e-3) / 1e12, bf16_tf, "tensor", "TFLOP/s"
+        else:
+            family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
+                w.B, w.H, w.T, w.d, w.mini_batch, w.dtype, w.mode)
+            kname = {"tensorcore": "ttt_linear_lag_kernel", "generic": "ttt_linear_generic_kernel"}[family]
+            achieved, peak, bound, unit = ab / (kernel_ms * 1e-3) / 1e9, hbm, "hbm", "GB/s"
         traffic = recorded_traffic(kname, w.name)
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": workload_config(w),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms,
-                         "kernel": kname},
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": ab, "algorithmic_flops_per_launch": af,
+                         "kernel_ms": kernel_ms, "kernel": kname},
             "cpu_baseline": cpu_base,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "kernel_impl": family,
-            "tflops_achieved": algorithmic_flops(w) / (kernel_ms * 1e-3) / 1e12,
+            "tflops_achieved": af / (kernel_ms * 1e-3) / 1e12,
+            "hbm_gbs_achieved": ab / (kernel_ms * 1e-3) / 1e9,
         }
         print(json.dumps(line), flush=True)
 
@@ -325,7 +377,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
-                    choices=[k for k, v in WORKLOADS.items() if v.kind == "linear"])
+                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048])
     ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore"], default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,

@@ -371,6 +371,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 ptx::ldsm_x4_t(ptx::smem_addr(s.E[pb][0]) + swz_chunk(row, chunk), ah[0], ah[1], ah[2], ah[3]);
                 ptx::ldsm_x4_t(ptx::smem_addr(s.E[pb][1]) + swz_chunk(row, chunk), al[0], al[1], al[2], al[3]);
             }
+            // The increment is formed in fresh accumulators and added to the state with fp32
+            // adds (round to nearest): the tensor-core accumulation does not round to nearest,
+            // and the state takes thousands of increments.
             {
                 const uint32_t xs = ptx::smem_addr(s.K[pslot]);
                 const int mi = lane >> 3;
@@ -379,14 +382,23 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     const int row = (mi & 1) * 8 + (lane & 7), chunk = 2 * jp + (mi >> 1);
                     uint32_t b0, b1, b2, b3;
                     ptx::ldsm_x4_t(xs + swz_chunk(row, chunk), b0, b1, b2, b3);
-                    ptx::mma_bf16(Wt[2 * jp], ah[0], ah[1], ah[2], ah[3], b0, b1);
-                    ptx::mma_bf16(Wt[2 * jp], al[0], al[1], al[2], al[3], b0, b1);
-                    ptx::mma_bf16(Wt[2 * jp + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
-                    ptx::mma_bf16(Wt[2 * jp + 1], al[0], al[1], al[2], al[3], b2, b3);
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                    ptx::mma_bf16(d0, ah[0], ah[1], ah[2], ah[3], b0, b1);
+                    ptx::mma_bf16(d0, al[0], al[1], al[2], al[3], b0, b1);
+                    ptx::mma_bf16(d1, ah[0], ah[1], ah[2], ah[3], b2, b3);
+                    ptx::mma_bf16(d1, al[0], al[1], al[2], al[3], b2, b3);
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        Wt[2 * jp][r] += d0[r];
+                        Wt[2 * jp + 1][r] += d1[r];
+                    }
                 }
                 // bias column: x~ has a 1 in it for every token
-                ptx::mma_bf16(Bt, ah[0], ah[1], ah[2], ah[3], ones, ones);
-                ptx::mma_bf16(Bt, al[0], al[1], al[2], al[3], ones, ones);
+                float db[4] = {0.f, 0.f, 0.f, 0.f};
+                ptx::mma_bf16(db, ah[0], ah[1], ah[2], ah[3], ones, ones);
+                ptx::mma_bf16(db, al[0], al[1], al[2], al[3], ones, ones);
+#pragma unroll
+                for (int r = 0; r < 4; r++) Bt[r] += db[r];
             }
             arrive1(&s.g_empty[pb], lane);
             arrive1(&s.in_empty[pslot], lane);
