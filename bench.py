@@ -166,10 +166,16 @@ def dist_setup():
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
+
+
+def weak_scaling_value(w, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own B*T tokens (all H heads)
+    per step; the step time is the max over ranks."""
+    return w.B * w.T * world / (ms_per_step * 1e-3)
 
 
 def dist_max(x: float, world: int) -> float:
@@ -316,7 +322,7 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
     kernel_ms = statistics.mean(per_launch_ms)
     tokens_per_step = w.B * w.T * world
-    value = tokens_per_step / (ms_per_step * 1e-3)
+    value = weak_scaling_value(w, world, ms_per_step)
 
     # end to end through the public API with pinned host buffers
     host_in = {k: v.pin_memory() for k, v in host.items() if v is not None}
