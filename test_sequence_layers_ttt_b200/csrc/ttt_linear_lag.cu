@@ -21,7 +21,9 @@
 //
 // Warp roles (480 threads):
 //   CH  warps 0-3   the chain: warp w owns output features [16w, 16w+16);
-//                   writes G_c and -eta G_c as bf16 hi/lo tiles
+//                   writes G_c and -eta G_c as bf16 hi/lo tiles and keeps G_c
+//                   as B fragments in registers (8x8 transposes, movmatrix);
+//                   reads the next chunk's W-free inputs early in each chunk
 //   WP  warps 4-7   the state: warp w keeps rows [16w, 16w+16) of W~^T (all
 //                   65 input columns, the last one the bias) as fp32 mma
 //                   accumulators; applies the update with G_{c-1}, then forms
@@ -456,20 +458,29 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 
         // per-chunk inputs, loaded one chunk ahead
         float R[2][4], gcv[8], c0v[2], etv[2];
-        uint4 mh, ml;
-        auto load_inputs = [&](int c) {
+        float ngcv[8], nc0v[2], netv[2];
+        uint4 mh, ml, nmh, nml;
+        auto load_pre = [&](int c) {
             const int b = c & 1;
             wait_use(&s.pre_full[b], c >> 1, abort_flag);
             const float4 g0 = s.gcbuf[b][w][lane][0], g1 = s.gcbuf[b][w][lane][1];
-            gcv[0] = g0.x; gcv[1] = g0.y; gcv[2] = g0.z; gcv[3] = g0.w;
-            gcv[4] = g1.x; gcv[5] = g1.y; gcv[6] = g1.z; gcv[7] = g1.w;
-            c0v[0] = s.c0[b][g];
-            c0v[1] = s.c0[b][g + 8];
-            etv[0] = s.etac[b][g];
-            etv[1] = s.etac[b][g + 8];
-            mh = s.mfrag[b][0][lane];
-            ml = s.mfrag[b][1][lane];
+            ngcv[0] = g0.x; ngcv[1] = g0.y; ngcv[2] = g0.z; ngcv[3] = g0.w;
+            ngcv[4] = g1.x; ngcv[5] = g1.y; ngcv[6] = g1.z; ngcv[7] = g1.w;
+            nc0v[0] = s.c0[b][g];
+            nc0v[1] = s.c0[b][g + 8];
+            netv[0] = s.etac[b][g];
+            netv[1] = s.etac[b][g + 8];
+            nmh = s.mfrag[b][0][lane];
+            nml = s.mfrag[b][1][lane];
             arrive1(&s.pre_empty[b], lane);
+        };
+        auto load_inputs = [&](int c) {
+            const int b = c & 1;
+#pragma unroll
+            for (int i = 0; i < 8; i++) gcv[i] = ngcv[i];
+            c0v[0] = nc0v[0]; c0v[1] = nc0v[1];
+            etv[0] = netv[0]; etv[1] = netv[1];
+            mh = nmh; ml = nml;
             wait_use(&s.p_full[b], c >> 1, abort_flag);
             const float4 p0 = s.pbuf[b][w][lane][0], p1 = s.pbuf[b][w][lane][1];
             R[0][0] = p0.x; R[0][1] = p0.y; R[0][2] = p0.z; R[0][3] = p0.w;
@@ -478,7 +489,10 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         };
 
         uint32_t gbh[4] = {0u, 0u, 0u, 0u}, gbl[4] = {0u, 0u, 0u, 0u};  // G_{c-1} as B fragments
-        if (n > 0) load_inputs(0);
+        if (n > 0) {
+            load_pre(0);
+            load_inputs(0);
+        }
         for (int c = 0; c < n; c++) {
             const int b = c & 1;
             float y[2][4];
@@ -494,6 +508,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 ptx::mma_bf16(y[0], ml.x, ml.y, ml.z, ml.w, gbh[0], gbh[1]);
                 ptx::mma_bf16(y[1], ml.x, ml.y, ml.z, ml.w, gbh[2], gbh[3]);
             }
+            if (c + 1 < n) load_pre(c + 1);
             const float* gcc = gcv;
             const float* c0c = c0v;
 
@@ -554,7 +569,17 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                         G[rh][nt][e] = fmaf(gx, rs, fmaf(xh, k2, k1));
                     }
             }
-            // G_c and -eta G_c (hi/lo) -> shared tiles; G_c back as B fragments
+            // G_c back as B fragments for the next chunk (8x8 transposes in registers)
+#pragma unroll
+            for (int rh = 0; rh < 2; rh++)
+#pragma unroll
+                for (int nt = 0; nt < 2; nt++) {
+                    uint32_t hi, lo;
+                    ptx::split_pair(G[rh][nt][0], G[rh][nt][1], hi, lo);
+                    gbh[2 * nt + rh] = ptx::movmatrix_t(hi);
+                    gbl[2 * nt + rh] = ptx::movmatrix_t(lo);
+                }
+            // G_c and -eta G_c (hi/lo) -> shared tiles for the state and output warps
             if (c >= 2) wait_use(&s.g_empty[b], (c >> 1) - 1, abort_flag);
 #pragma unroll
             for (int rh = 0; rh < 2; rh++)
@@ -569,12 +594,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     *reinterpret_cast<uint32_t*>(s.E[b][0] + off) = ehi;
                     *reinterpret_cast<uint32_t*>(s.E[b][1] + off) = elo;
                 }
-            __syncwarp();
-            {
-                const int mi = lane >> 3, row = (mi & 1) * 8 + (lane & 7), chunk = 2 * w + (mi >> 1);
-                ptx::ldsm_x4_t(ptx::smem_addr(s.G[b][0]) + swz_chunk(row, chunk), gbh[0], gbh[1], gbh[2], gbh[3]);
-                ptx::ldsm_x4_t(ptx::smem_addr(s.G[b][1]) + swz_chunk(row, chunk), gbl[0], gbl[1], gbl[2], gbl[3]);
-            }
+            __syncwarp();  // every lane's tile stores before the hand-off
             if (lane == 0) ptx::mbar_arrive(&s.g_full[b]);
             if (c + 1 < n) load_inputs(c + 1);
         }
