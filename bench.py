@@ -283,7 +283,8 @@ def run_ours(args, world, rank, local):
                                        ln_eps=w.ln_eps, **kw)
 
         def step():
-            call(g, Z=Z, W1_T=state["W1"], b1_T=state["b1"], W2_T=state["W2"], b2_T=state["b2"],
+            call(g, impl=args.kernel, Z=Z, W1_T=state["W1"], b1_T=state["b1"], W2_T=state["W2"],
+                 b2_T=state["b2"],
                  stream=stream)
     else:
         keys = KEYS
@@ -347,7 +348,9 @@ def run_ours(args, world, rank, local):
         ab = algorithmic_bytes(w)
         af = algorithmic_flops(w)
         if w.kind == "mlp":
-            family, kname = "generic", "ttt_mlp_generic_kernel"
+            family = args.kernel if args.kernel != "auto" else ttt.mlp_pick_impl(
+                w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype)
+            kname = {"tensorcore": "ttt_mlp_tc_kernel", "generic": "ttt_mlp_generic_kernel"}[family]
             achieved, peak, bound, unit = af / (kernel_ms * 1e-3) / 1e12, bf16_tf, "tensor", "TFLOP/s"
         else:
             family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(

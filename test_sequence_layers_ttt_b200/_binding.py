@@ -46,6 +46,10 @@ lib.ttt_linear_forward_impl.restype = _I
 lib.ttt_linear_forward_impl.argtypes = [_I] * 7 + [_F] + [_P] * 11 + [_I, _P]
 lib.ttt_mlp_forward.restype = _I
 lib.ttt_mlp_forward.argtypes = [_I] * 7 + [_F] + [_P] * 15 + [_P]
+lib.ttt_mlp_forward_impl.restype = _I
+lib.ttt_mlp_forward_impl.argtypes = [_I] * 7 + [_F] + [_P] * 15 + [_I, _P]
+lib.ttt_mlp_pick_impl.restype = _I
+lib.ttt_mlp_pick_impl.argtypes = [_I] * 7
 lib.ttt_status_string.restype = ctypes.c_char_p
 lib.ttt_status_string.argtypes = [_I]
 lib.ttt_abi_version.restype = _I
@@ -59,6 +63,13 @@ def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
     code = lib.ttt_linear_pick_impl(B, H, T, d, mini_batch,
                                     TTT_BF16 if qkv_dtype in ("bf16", torch.bfloat16) else TTT_F32,
                                     _mode_code(mode))
+    return {0: "none", 1: "generic", 2: "tensorcore"}[code]
+
+
+def mlp_pick_impl(B, H, T, d, hidden, mini_batch, qkv_dtype) -> str:
+    """Kernel family the library's AUTO dispatch runs for these TTT-MLP arguments."""
+    code = lib.ttt_mlp_pick_impl(B, H, T, d, hidden, mini_batch,
+                                 TTT_BF16 if qkv_dtype in ("bf16", torch.bfloat16) else TTT_F32)
     return {0: "none", 1: "generic", 2: "tensorcore"}[code]
 
 
@@ -162,8 +173,8 @@ def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *
 
 
 def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
-                    mini_batch: int = 16, ln_eps: float = 1e-6, Z=None, W1_T=None, b1_T=None,
-                    W2_T=None, b2_T=None, stream=None):
+                    mini_batch: int = 16, ln_eps: float = 1e-6, impl: str = "auto", Z=None,
+                    W1_T=None, b1_T=None, W2_T=None, b2_T=None, stream=None):
     """TTT-MLP forward scan (see include/ttt.h).  Returns (Z, W1_T, b1_T, W2_T, b2_T)."""
     rt = _HostRoundTrip([Q, K, V, eta, W1_0])
     Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta = (
@@ -181,10 +192,10 @@ def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
     b1_T = torch.empty((B, H, hid), **f32) if b1_T is None else b1_T
     W2_T = torch.empty((B, H, hid, d), **f32) if W2_T is None else W2_T
     b2_T = torch.empty((B, H, d), **f32) if b2_T is None else b2_T
-    st = lib.ttt_mlp_forward(
+    st = lib.ttt_mlp_forward_impl(
         B, H, T, d, hid, int(mini_batch), _dtype_code(Q), float(ln_eps), _ptr(Q), _ptr(K),
         _ptr(V), _ptr(eta), _ptr(W1_0), _ptr(b1_0), _ptr(W2_0), _ptr(b2_0), _ptr(ln_gamma),
-        _ptr(ln_beta), _ptr(Z), _ptr(W1_T), _ptr(b1_T), _ptr(W2_T), _ptr(b2_T),
+        _ptr(ln_beta), _ptr(Z), _ptr(W1_T), _ptr(b1_T), _ptr(W2_T), _ptr(b2_T), IMPLS[impl],
         _stream_handle(dev, stream))
     _check(st)
     return rt.to_host((Z, W1_T, b1_T, W2_T, b2_T))

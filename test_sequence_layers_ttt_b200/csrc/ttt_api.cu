@@ -153,18 +153,48 @@ ttt_status ttt_linear_forward(int B, int H, int T, int d, int mini_batch, ttt_dt
                                    W0, b0, ln_gamma, ln_beta, Z, W_T, b_T, TTT_IMPL_AUTO, stream);
 }
 
+ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini_batch,
+                                ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
+                                const void* V, const float* eta, const float* W1_0, const float* b1_0,
+                                const float* W2_0, const float* b2_0, const float* ln_gamma,
+                                const float* ln_beta, float* Z, float* W1_T, float* b1_T, float* W2_T,
+                                float* b2_T, ttt_impl impl, ttt_stream_t stream) {
+    MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1_0, b1_0,
+              W2_0, b2_0, ln_gamma, ln_beta, Z, W1_T, b1_T, W2_T, b2_T};
+    ttt_status st = validate_mlp(a);
+    if (st != TTT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (impl) {
+        case TTT_IMPL_AUTO:
+            if (ttt::mlp_tc_supports(a)) return finish(ttt::launch_mlp_tc(a, s), s);
+            return finish(ttt::launch_mlp_generic(a, s), s);
+        case TTT_IMPL_GENERIC:
+            return finish(ttt::launch_mlp_generic(a, s), s);
+        case TTT_IMPL_TENSORCORE:
+            if (!ttt::mlp_tc_supports(a)) return TTT_ERR_UNSUPPORTED;
+            return finish(ttt::launch_mlp_tc(a, s), s);
+        default:
+            return TTT_ERR_UNSUPPORTED;
+    }
+}
+
+ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch, ttt_dtype qkv_dtype) {
+    MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, 1e-6f, nullptr, nullptr, nullptr, nullptr,
+              nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+              nullptr};
+    if (ttt::mlp_tc_supports(a)) return TTT_IMPL_TENSORCORE;
+    return ttt::mlp_generic_supports(a) ? TTT_IMPL_GENERIC : TTT_IMPL_AUTO;
+}
+
 ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batch,
                            ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
                            const void* V, const float* eta, const float* W1_0, const float* b1_0,
                            const float* W2_0, const float* b2_0, const float* ln_gamma,
                            const float* ln_beta, float* Z, float* W1_T, float* b1_T, float* W2_T,
                            float* b2_T, ttt_stream_t stream) {
-    MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1_0, b1_0,
-              W2_0, b2_0, ln_gamma, ln_beta, Z, W1_T, b1_T, W2_T, b2_T};
-    ttt_status st = validate_mlp(a);
-    if (st != TTT_OK) return st;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return finish(ttt::launch_mlp_generic(a, s), s);
+    return ttt_mlp_forward_impl(B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1_0,
+                                b1_0, W2_0, b2_0, ln_gamma, ln_beta, Z, W1_T, b1_T, W2_T, b2_T,
+                                TTT_IMPL_AUTO, stream);
 }
 
 const char* ttt_status_string(ttt_status status) {

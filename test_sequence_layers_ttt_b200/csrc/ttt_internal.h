@@ -35,6 +35,9 @@ cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream);
 bool mlp_generic_supports(const MlpArgs& a);
 cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);
 
+bool mlp_tc_supports(const MlpArgs& a);
+cudaError_t launch_mlp_tc(const MlpArgs& a, cudaStream_t stream);
+
 // Device-side error word set by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_device_error(unsigned int* out);
 

@@ -146,6 +146,15 @@ def test_pick_impl_is_a_host_query():
     assert f(2, 32, 32768, 64, 16, 0, 0) in (1, 2)
 
 
+def test_mlp_pick_impl_is_a_host_query():
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "bf16") == "tensorcore"
+    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "f32") == "generic"
+    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 32, "bf16") == "generic"
+    assert ttt.mlp_pick_impl(4, 12, 8200, 64, 256, 16, "bf16") == "generic"
+    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 128, 16, "bf16") == "none"
+
+
 def test_empty_sequence_allows_null_token_buffers_but_not_state():
     p = [fake(k) for k in range(11)]
     for i in (0, 1, 2, 3, 8):

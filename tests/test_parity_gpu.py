@@ -247,10 +247,10 @@ def test_linear_host_buffers_end_to_end(ttt):
 
 # ------------------------------------------------------------------ TTT-MLP
 
-def gpu_mlp(ttt, w, inp, mini_batch=None):
+def gpu_mlp(ttt, w, inp, mini_batch=None, impl="auto"):
     g = to_cuda(inp)
     out = ttt.ttt_mlp_forward(*(g[k] for k in MLP_KEYS), mini_batch=mini_batch or w.mini_batch,
-                              ln_eps=w.ln_eps)
+                              ln_eps=w.ln_eps, impl=impl)
     torch.cuda.synchronize()
     return [o.cpu().numpy() for o in out]
 
@@ -259,8 +259,8 @@ def oracle_mlp(w, inp, mini_batch=None):
     return oracle.ttt_mlp(*(inp[k] for k in MLP_KEYS), mini_batch or w.mini_batch, w.ln_eps)
 
 
-def compare_mlp(ttt, w, inp, mini_batch=None, pairs=None):
-    out = gpu_mlp(ttt, w, inp, mini_batch)
+def compare_mlp(ttt, w, inp, mini_batch=None, pairs=None, impl="auto"):
+    out = gpu_mlp(ttt, w, inp, mini_batch, impl)
     if pairs is not None:
         ref = oracle_mlp(w, select_heads(inp, pairs), mini_batch)
         out = [np.stack([o[bb, hh] for bb, hh in pairs])[None] for o in out]
@@ -291,5 +291,67 @@ def test_mlp_f32_inputs(ttt):
 
 
 def test_mlp_full_sampled_heads(ttt):
+    """The benchmarked launch (tensor-core family): all 48 scans of 8k tokens on
+    the GPU, three checked end to end against the oracle."""
     w = WORKLOADS["mlp_8k"]
+    assert ttt.mlp_pick_impl(w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype) == "tensorcore"
     compare_mlp(ttt, w, make_inputs(w, 0), pairs=[(0, 0), (2, 7), (3, 11)])
+
+
+@pytest.mark.parametrize("T", [16, 48, 256, 1024])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_mlp_tensorcore_vs_oracle(ttt, T, seed):
+    """Several chunks, all heads of a small batch, the tensor-core family explicitly."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=2, H=3, T=T)
+    compare_mlp(ttt, w, make_inputs(w, seed), impl="tensorcore")
+
+
+def test_mlp_generic_explicit_on_the_tensorcore_shape(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=128)
+    compare_mlp(ttt, w, make_inputs(w, 4), impl="generic")
+
+
+def test_mlp_tensorcore_matches_generic(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=512)
+    inp = make_inputs(w, 9)
+    tc = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    ge = gpu_mlp(ttt, w, inp, impl="generic")
+    for name, a, b in zip(("Z", "W1_T", "b1_T", "W2_T", "b2_T"), tc, ge):
+        assert_close(a, b.astype(np.float64), 1e-3, f"{name} tensorcore vs generic",
+                     denom=max(rms(b), 1e-3))
+
+
+def test_mlp_tensorcore_continuation(ttt):
+    """Two calls split at a mini-batch boundary, the state carried through the
+    final-state buffers, equal one call up to rounding."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=256)
+    inp = make_inputs(w, 5)
+    full = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    half = w.with_shape(T=128)
+    first = {k: (v[:, :, :128].contiguous() if k in ("Q", "K", "V", "eta") else v) for k, v in inp.items()}
+    out1 = gpu_mlp(ttt, half, first, impl="tensorcore")
+    second = {k: (v[:, :, 128:].contiguous() if k in ("Q", "K", "V", "eta") else v) for k, v in inp.items()}
+    for k, o in zip(("W1_0", "b1_0", "W2_0", "b2_0"), out1[1:]):
+        second[k] = torch.from_numpy(o)
+    out2 = gpu_mlp(ttt, half, second, impl="tensorcore")
+    Z = np.concatenate([out1[0], out2[0]], axis=2)
+    assert_close(Z, full[0].astype(np.float64), 1e-4, "Z continuation")
+    for name, a, b in zip(("W1_T", "b1_T", "W2_T", "b2_T"), out2[1:], full[1:]):
+        assert_close(a, b.astype(np.float64), 1e-4, name, denom=max(rms(b), 1e-3))
+
+
+def test_mlp_tensorcore_is_deterministic(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=256)
+    inp = make_inputs(w, 6)
+    a = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    b = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("kw", [dict(T=40), dict(dtype="f32", T=64)])
+def test_mlp_tensorcore_unsupported_shapes(ttt, kw):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=1, **kw)
+    with pytest.raises(ttt.TTTError) as ei:
+        gpu_mlp(ttt, w, make_inputs(w, 0), impl="tensorcore")
+    assert ei.value.status == 6
