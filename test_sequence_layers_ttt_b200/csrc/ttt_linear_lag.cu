@@ -34,6 +34,9 @@
 //   PB  warp 14     M_c and A_c (16 x 16 tensor-core products, eta folded in)
 // Every product with an fp32 operand splits it into bf16 hi + lo terms
 // (relative error below 2^-15); bf16 inputs are exact; accumulation is fp32.
+// The W-free inputs run up to NPRE chunks ahead in a ring, and Q~W~ is handed
+// to the output warps through four buffers, so the slower output path does
+// not hold back the chain's inputs.
 // Hand-offs between roles are mbarriers with bounded waits: after about a
 // second without progress the kernel records an error word, stops waiting and
 // drains its TMA loads (outputs undefined; TTT_ERR_TIMEOUT with TTT_CHECK=1).
@@ -53,6 +56,7 @@ namespace {
 
 constexpr int D = 64;
 constexpr int NS = 8;            // TMA ring stages
+constexpr int NPRE = 8;          // ring of the chain's and output's W-free inputs
 constexpr int kCH = 4, kWP = 4, kOW = 4;
 constexpr int kWarpWP0 = kCH, kWarpOW0 = kCH + kWP, kWarpPR = kCH + kWP + kOW;
 constexpr int kWarpPA = kWarpPR + 1, kWarpPB = kWarpPR + 2;
@@ -70,19 +74,19 @@ struct LagSmem {
     unsigned char G[2][2][TILE];            // [buf][hi, lo] G_c, swizzled [tok][out] bf16
     unsigned char E[2][2][TILE];            // [buf][hi, lo] -eta G_c, same layout
     float4 pbuf[2][kCH][32][2];             // [buf][w][lane]: P_c fragments (8 floats)
-    float4 qwbuf[2][kCH][32][2];            // same for Q~_c W~_c
-    float4 gcbuf[2][kCH][32][2];            // g * (x + beta - v) in chain fragment order
-    uint4 mfrag[2][2][32];                  // [buf][hi, lo] -M_c as A fragments
-    uint4 afrag[2][2][32];                  // [buf][hi, lo] -A_c as A fragments
-    float c0[2][kChunk];                    // row sums of g * c'
-    float etac[2][kChunk];                  // eta of the chunk, for the chain
+    float4 qwbuf[4][kCH][32][2];            // same for Q~_c W~_c, [c % 4]
+    float4 gcbuf[NPRE][kCH][32][2];         // g * (x + beta - v) in chain fragment order
+    uint4 mfrag[NPRE][2][32];               // [c % NPRE][hi, lo] -M_c as A fragments
+    uint4 afrag[NPRE][2][32];               // [c % NPRE][hi, lo] -A_c as A fragments
+    float c0[NPRE][kChunk];                 // row sums of g * c'
+    float etac[NPRE][kChunk];               // eta of the chunk, for the chain
     alignas(128) float eta[NS][32];
     float red_ch[2][kChunk][5][4];          // [buf][tok][sum][warp]
     float red_ow[2][kChunk][12];            // [buf][tok][2 sums x 4 warps + pad]
     float gam[D], bet[D];
     uint64_t in_full[NS], in_empty[NS];
-    uint64_t pre_full[2], pre_empty[2], p_full[2], p_empty[2];
-    uint64_t g_full[2], g_empty[2], qw_full[2], qw_empty[2];
+    uint64_t pre_full[NPRE], pre_empty[NPRE], p_full[2], p_empty[2];
+    uint64_t g_full[2], g_empty[2], qw_full[4], qw_empty[4];
     int abort_flag;
 };
 
@@ -140,15 +144,19 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             ptx::mbar_init(&s.in_full[i], 1);
             ptx::mbar_init(&s.in_empty[i], 2 + kWP + kOW);  // PA, PB, WP, OW
         }
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < NPRE; i++) {
             ptx::mbar_init(&s.pre_full[i], 2);            // PA, PB
             ptx::mbar_init(&s.pre_empty[i], kCH + kOW);
+        }
+        for (int i = 0; i < 2; i++) {
             ptx::mbar_init(&s.p_full[i], kWP);
             ptx::mbar_init(&s.p_empty[i], kCH);
             ptx::mbar_init(&s.g_full[i], kCH);
             ptx::mbar_init(&s.g_empty[i], kWP + kOW);
             ptx::mbar_init(&s.qw_full[i], kWP);
             ptx::mbar_init(&s.qw_empty[i], kOW);
+            ptx::mbar_init(&s.qw_full[i + 2], kWP);
+            ptx::mbar_init(&s.qw_empty[i + 2], kOW);
         }
         ptx::fence_mbar_init();
     }
@@ -190,9 +198,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     // ================================================================ PA: g * (x + beta - v), row sums
     if (warp == kWarpPA) {
         for (int c = 0; c < n; c++) {
-            const int slot = c % NS, b = c & 1;
+            const int slot = c % NS, b = c % NPRE;
             wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
-            if (c >= 2) wait_use(&s.pre_empty[b], (c >> 1) - 1, abort_flag);
+            if (c >= NPRE) wait_use(&s.pre_empty[b], c / NPRE - 1, abort_flag);
             float rs0 = 0.f, rs1 = 0.f;  // row g, row g + 8
 #pragma unroll
             for (int w = 0; w < kCH; w++) {
@@ -231,9 +239,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     // ================================================================ PB: M_c and A_c
     if (warp == kWarpPB) {
         for (int c = 0; c < n; c++) {
-            const int slot = c % NS, b = c & 1;
+            const int slot = c % NS, b = c % NPRE;
             wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
-            if (c >= 2) wait_use(&s.pre_empty[b], (c >> 1) - 1, abort_flag);
+            if (c >= NPRE) wait_use(&s.pre_empty[b], c / NPRE - 1, abort_flag);
             const uint32_t xs = ptx::smem_addr(s.K[slot]);
             const uint32_t qs = ptx::smem_addr(s.Q[slot]);
             const int mi = lane >> 3;
@@ -417,8 +425,8 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             }
             // ---- Q~_j W~_j for the output warps
             {
-                const int qb = j & 1;
-                if (j >= 2) wait_use(&s.qw_empty[qb], (j >> 1) - 1, abort_flag);
+                const int qb = j & 3;
+                if (j >= 4) wait_use(&s.qw_empty[qb], (j >> 2) - 1, abort_flag);
                 product(ptx::smem_addr(s.Q[j % NS]), s.qwbuf[qb][w][lane]);
                 arrive1(&s.qw_full[qb], lane);
             }
@@ -461,8 +469,8 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         float ngcv[8], nc0v[2], netv[2];
         uint4 mh, ml, nmh, nml;
         auto load_pre = [&](int c) {
-            const int b = c & 1;
-            wait_use(&s.pre_full[b], c >> 1, abort_flag);
+            const int b = c % NPRE;
+            wait_use(&s.pre_full[b], c / NPRE, abort_flag);
             const float4 g0 = s.gcbuf[b][w][lane][0], g1 = s.gcbuf[b][w][lane][1];
             ngcv[0] = g0.x; ngcv[1] = g0.y; ngcv[2] = g0.z; ngcv[3] = g0.w;
             ngcv[4] = g1.x; ngcv[5] = g1.y; ngcv[6] = g1.z; ngcv[7] = g1.w;
@@ -616,16 +624,16 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         for (int c = 0; c < n; c++) {
             const int b = c & 1, slot = c % NS;
             float z[2][4];
-            wait_use(&s.qw_full[b], c >> 1, abort_flag);
+            wait_use(&s.qw_full[c & 3], c >> 2, abort_flag);
             {
-                const float4 p0 = s.qwbuf[b][w][lane][0], p1 = s.qwbuf[b][w][lane][1];
+                const float4 p0 = s.qwbuf[c & 3][w][lane][0], p1 = s.qwbuf[c & 3][w][lane][1];
                 z[0][0] = p0.x; z[0][1] = p0.y; z[0][2] = p0.z; z[0][3] = p0.w;
                 z[1][0] = p1.x; z[1][1] = p1.y; z[1][2] = p1.z; z[1][3] = p1.w;
             }
-            arrive1(&s.qw_empty[b], lane);
-            wait_use(&s.pre_full[b], c >> 1, abort_flag);
-            const uint4 ah = s.afrag[b][0][lane], al = s.afrag[b][1][lane];
-            arrive1(&s.pre_empty[b], lane);
+            arrive1(&s.qw_empty[c & 3], lane);
+            wait_use(&s.pre_full[c % NPRE], c / NPRE, abort_flag);
+            const uint4 ah = s.afrag[c % NPRE][0][lane], al = s.afrag[c % NPRE][1][lane];
+            arrive1(&s.pre_empty[c % NPRE], lane);
             wait_use(&s.g_full[b], c >> 1, abort_flag);
             {
                 const int mi = lane >> 3, row = (mi & 1) * 8 + (lane & 7), chunk = 2 * w + (mi >> 1);
