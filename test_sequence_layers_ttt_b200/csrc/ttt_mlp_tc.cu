@@ -60,6 +60,21 @@ struct MlpTcSmem {
     alignas(16) float eta[kChunk];
 };
 
+// GELU (tanh form) through the logistic identity 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u)),
+// u = sqrt(2/pi) (x + 0.044715 x^3); returns gelu(x) and keeps sig for the derivative
+__device__ __forceinline__ float gelu_sig(float x, float& sig) {
+    const float c = 0.7978845608028654f;
+    const float u = c * fmaf(0.044715f * x, x * x, x);
+    sig = __fdividef(1.f, 1.f + __expf(-2.f * u));
+    return x * sig;
+}
+// d/dx [x sig(2u)] = sig + 2 x u' sig (1 - sig)
+__device__ __forceinline__ float gelu_prime_sig(float x, float sig) {
+    const float c = 0.7978845608028654f;
+    const float du = c * fmaf(3.f * 0.044715f * x, x, 1.f);
+    return fmaf(2.f * x * du * sig, 1.f - sig, sig);
+}
+
 // fp32 state indexing: 8-float groups of a row XOR-swizzled by the row's low bits
 __device__ __forceinline__ int w1i(int hid, int in) { return hid * D + ((((in >> 3) ^ (hid & 7))) << 3) + (in & 7); }
 __device__ __forceinline__ int w2i(int out, int hid) { return out * HID + ((((hid >> 3) ^ (out & 7))) << 3) + (hid & 7); }
@@ -190,7 +205,7 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
 
         // ================================================= phase 1: [X; Q] W1 + b1, H = GELU(Z1); A; -eta X
         // warp w: hidden units [16w, 16w + 16)
-        float z1[2][4], zq[2][4];
+        float z1[2][4], zq[2][4], sg1[2][4];
         {
 #pragma unroll
             for (int nt = 0; nt < 2; nt++) {
@@ -222,7 +237,7 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
             for (int nt = 0; nt < 2; nt++) {
                 float hv[4];
 #pragma unroll
-                for (int r = 0; r < 4; r++) hv[r] = gelu_tanh(z1[nt][r]);
+                for (int r = 0; r < 4; r++) hv[r] = gelu_sig(z1[nt][r], sg1[nt][r]);
                 store_pairs(s.Hh[p], s.Hl[p], g, 16 * (warp & 3) + 8 * nt + 2 * t, hv);
             }
         }
@@ -339,7 +354,7 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
 #pragma unroll
             for (int nt = 0; nt < 2; nt++) {
 #pragma unroll
-                for (int r = 0; r < 4; r++) acc[nt][r] *= gelu_tanh_prime(z1[nt][r]);
+                for (int r = 0; r < 4; r++) acc[nt][r] *= gelu_prime_sig(z1[nt][r], sg1[nt][r]);
                 store_pairs(s.G1h[p], s.G1l[p], g, 16 * (warp & 3) + 8 * nt + 2 * t, acc[nt]);
             }
         }
@@ -357,9 +372,9 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
             mma3(zq[1], ah, al, bh[2], bh[3], bl[2], bl[3]);
 #pragma unroll
             for (int nt = 0; nt < 2; nt++) {
-                float hv[4];
+                float hv[4], sq;
 #pragma unroll
-                for (int r = 0; r < 4; r++) hv[r] = gelu_tanh(zq[nt][r]);
+                for (int r = 0; r < 4; r++) hv[r] = gelu_sig(zq[nt][r], sq);
                 store_pairs(s.Hqh[p], s.Hql[p], g, 16 * (warp & 3) + 8 * nt + 2 * t, hv);
             }
         }
