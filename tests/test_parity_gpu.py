@@ -349,6 +349,32 @@ def test_mlp_tensorcore_is_deterministic(ttt):
         np.testing.assert_array_equal(x, y)
 
 
+def test_mlp_host_buffers_end_to_end(ttt):
+    """CPU tensors in, CPU tensors out through the public call (the bench's
+    end-to-end path), equal to the device-resident call."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=128)
+    inp = make_inputs(w, 7)
+    host = ttt.ttt_mlp_forward(*(inp[k] for k in MLP_KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps)
+    assert all(o.device.type == "cpu" for o in host)
+    dev = gpu_mlp(ttt, w, inp)
+    for a, b in zip(host, dev):
+        np.testing.assert_array_equal(a.numpy(), b)
+
+
+@pytest.mark.parametrize("impl", ["tensorcore", "generic"])
+def test_mlp_in_place_state(ttt, impl):
+    """Final-state buffers that are the initial-state buffers (in-place update)."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=64)
+    inp = make_inputs(w, 8)
+    ref = gpu_mlp(ttt, w, inp, impl=impl)
+    g = to_cuda(inp)
+    ttt.ttt_mlp_forward(*(g[k] for k in MLP_KEYS), mini_batch=w.mini_batch, ln_eps=w.ln_eps, impl=impl,
+                        W1_T=g["W1_0"], b1_T=g["b1_0"], W2_T=g["W2_0"], b2_T=g["b2_0"])
+    torch.cuda.synchronize()
+    for name, r in zip(("W1_0", "b1_0", "W2_0", "b2_0"), ref[1:]):
+        np.testing.assert_array_equal(g[name].cpu().numpy(), r)
+
+
 @pytest.mark.parametrize("kw", [dict(T=40), dict(dtype="f32", T=64)])
 def test_mlp_tensorcore_unsupported_shapes(ttt, kw):
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=1, **kw)
