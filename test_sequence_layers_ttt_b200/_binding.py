@@ -139,11 +139,83 @@ class _HostRoundTrip:
         return tuple(host)
 
 
+_STREAMS = {}
+
+
+def _side_streams(dev: torch.device, n: int):
+    key = (dev.index, n)
+    if key not in _STREAMS:
+        _STREAMS[key] = [torch.cuda.Stream(device=dev) for _ in range(n)]
+    return _STREAMS[key]
+
+
+def _head_groups(B: int, H: int, n: int):
+    """(batch, first head, end head) groups of about B*H/n scans each."""
+    per = max(1, -(-(B * H) // n))
+    return [(b, h0, min(H, h0 + per)) for b in range(B) for h0 in range(0, H, per)]
+
+
+def _pinned(t):
+    return None if t is None else (t if t.is_pinned() else t.pin_memory())
+
+
+def _host_pipeline(device_call, per_scan: dict, per_head: dict, out_shapes: dict, n_groups: int = 8):
+    """End-to-end path for host tensors: the (batch, head) scans are independent,
+    so they are cut into groups, and each group's copies in, scan and copies out
+    run on their own stream; one group's transfers overlap the others' scans and
+    the two copy directions overlap each other.  Results land in pinned host
+    tensors; the call returns when every copy back has finished."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    any_t = next(t for t in per_scan.values() if t is not None)
+    B, H = any_t.shape[:2]
+    per_scan = {k: _pinned(t) for k, t in per_scan.items()}
+    per_head = {k: _pinned(t) for k, t in per_head.items()}
+    outs = {k: (None if shp is None else torch.empty(shp, dtype=torch.float32, pin_memory=True))
+            for k, shp in out_shapes.items()}
+    groups = _head_groups(B, H, n_groups)
+    streams = _side_streams(dev, min(n_groups, len(groups)))
+    current = torch.cuda.current_stream(dev)
+    for s in streams:
+        s.wait_stream(current)
+    for i, (b, h0, h1) in enumerate(groups):
+        s = streams[i % len(streams)]
+        with torch.cuda.stream(s):
+            args = {k: (None if t is None else t[b:b + 1, h0:h1].to(dev, non_blocking=True))
+                    for k, t in per_scan.items()}
+            args.update({k: (None if t is None else t[h0:h1].to(dev, non_blocking=True))
+                         for k, t in per_head.items()})
+            res = device_call(args, s)
+            for (k, host), r in zip(outs.items(), res):
+                if host is not None:
+                    host[b:b + 1, h0:h1].copy_(r, non_blocking=True)
+    for s in streams:
+        s.synchronize()
+    return tuple(outs.values())
+
+
+def _on_host(*ts) -> bool:
+    return all(t is None or t.device.type == "cpu" for t in ts)
+
+
 def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *,
                        mini_batch: int = 16, mode="ln", ln_eps: float = 1e-6, impl: str = "auto",
                        Z=None, W_T=None, b_T=None, stream=None
                        ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
-    """TTT-Linear forward scan (see include/ttt.h).  Returns (Z, W_T, b_T)."""
+    """TTT-Linear forward scan (see include/ttt.h).  Returns (Z, W_T, b_T).
+    Host (CPU) tensors in, host tensors out when every input is on the host."""
+    if (_on_host(Q, K, V, eta, W0, b0, ln_gamma, ln_beta) and Z is None and W_T is None and b_T is None
+            and stream is None and Q.dim() == 4 and Q.shape[0] * Q.shape[1] > 1 and Q.shape[2] > 0):
+        B, H, T, d = Q.shape
+        plain = _mode_code(mode) == TTT_PLAIN
+
+        def run(a, s):
+            return ttt_linear_forward(a["Q"], a["K"], a["V"], a["eta"], a["W0"], a["b0"], a["ln_gamma"],
+                                      a["ln_beta"], mini_batch=mini_batch, mode=mode, ln_eps=ln_eps,
+                                      impl=impl, stream=s)
+
+        return _host_pipeline(run, dict(Q=Q, K=K, V=V, eta=eta, W0=W0, b0=b0),
+                              dict(ln_gamma=ln_gamma, ln_beta=ln_beta),
+                              dict(Z=(B, H, T, d), W_T=(B, H, d, d), b_T=None if plain else (B, H, d)))
     rt = _HostRoundTrip([Q, K, V, eta, W0])
     Q, K, V, eta, W0, b0, ln_gamma, ln_beta = (
         rt.to_device(x) for x in (Q, K, V, eta, W0, b0, ln_gamma, ln_beta))
@@ -175,7 +247,23 @@ def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *
 def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
                     mini_batch: int = 16, ln_eps: float = 1e-6, impl: str = "auto", Z=None,
                     W1_T=None, b1_T=None, W2_T=None, b2_T=None, stream=None):
-    """TTT-MLP forward scan (see include/ttt.h).  Returns (Z, W1_T, b1_T, W2_T, b2_T)."""
+    """TTT-MLP forward scan (see include/ttt.h).  Returns (Z, W1_T, b1_T, W2_T, b2_T).
+    Host (CPU) tensors in, host tensors out when every input is on the host."""
+    if (_on_host(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta)
+            and all(o is None for o in (Z, W1_T, b1_T, W2_T, b2_T)) and stream is None and Q.dim() == 4
+            and Q.shape[0] * Q.shape[1] > 1 and Q.shape[2] > 0):
+        B, H, T, d = Q.shape
+        hid = W1_0.shape[-1]
+
+        def run(a, s):
+            return ttt_mlp_forward(a["Q"], a["K"], a["V"], a["eta"], a["W1_0"], a["b1_0"], a["W2_0"],
+                                   a["b2_0"], a["ln_gamma"], a["ln_beta"], mini_batch=mini_batch,
+                                   ln_eps=ln_eps, impl=impl, stream=s)
+
+        return _host_pipeline(run, dict(Q=Q, K=K, V=V, eta=eta, W1_0=W1_0, b1_0=b1_0, W2_0=W2_0, b2_0=b2_0),
+                              dict(ln_gamma=ln_gamma, ln_beta=ln_beta),
+                              dict(Z=(B, H, T, d), W1_T=(B, H, d, hid), b1_T=(B, H, hid),
+                                   W2_T=(B, H, hid, d), b2_T=(B, H, d)))
     rt = _HostRoundTrip([Q, K, V, eta, W1_0])
     Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta = (
         rt.to_device(x) for x in (Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta))

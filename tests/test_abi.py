@@ -146,6 +146,15 @@ def test_pick_impl_is_a_host_query():
     assert f(2, 32, 32768, 64, 16, 0, 0) in (1, 2)
 
 
+@pytest.mark.parametrize("B,H,n", [(1, 3, 8), (2, 32, 8), (4, 12, 8), (2, 5, 8), (1, 1, 8), (3, 7, 4)])
+def test_host_pipeline_groups_cover_every_scan_once(B, H, n):
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+    groups = ttt._head_groups(B, H, n)
+    seen = [(b, h) for b, h0, h1 in groups for h in range(h0, h1)]
+    assert sorted(seen) == [(b, h) for b in range(B) for h in range(H)]
+    assert all(h1 > h0 for _, h0, h1 in groups)
+
+
 def test_mlp_pick_impl_is_a_host_query():
     from test_sequence_layers_ttt_b200 import _binding as ttt
     assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "bf16") == "tensorcore"

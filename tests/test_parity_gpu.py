@@ -245,6 +245,25 @@ def test_linear_host_buffers_end_to_end(ttt):
     np.testing.assert_array_equal(Wh.numpy(), Wd)
 
 
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_linear_host_pipeline_uneven_groups(ttt, mode):
+    """The host path cuts the scans into groups on several streams; groups of
+    unequal size, both modes, and the result equals the device call bit for bit."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=5, T=64)
+    if mode == "plain":
+        w = w.with_shape(mode=MODE_PLAIN)
+    inp = make_inputs(w, 3)
+    plain = mode == "plain"
+    host = ttt.ttt_linear_forward(inp["Q"], inp["K"], inp["V"], inp["eta"], inp["W0"],
+                                  None if plain else inp["b0"], None if plain else inp["gamma"],
+                                  None if plain else inp["beta"], mode=mode)
+    dev = gpu_linear(ttt, w, inp)
+    np.testing.assert_array_equal(host[0].numpy(), dev[0])
+    np.testing.assert_array_equal(host[1].numpy(), dev[1])
+    if not plain:
+        np.testing.assert_array_equal(host[2].numpy(), dev[2])
+
+
 # ------------------------------------------------------------------ TTT-MLP
 
 def gpu_mlp(ttt, w, inp, mini_batch=None, impl="auto"):
