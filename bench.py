@@ -79,10 +79,20 @@ def load_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "ttt_linear_lag_kernel": ("ttt_linear_lag.cu", "ptx.cuh", "common.cuh", "tma_host.h", "ttt_internal.h"),
+    "ttt_linear_generic_kernel": ("ttt_linear_generic.cu", "common.cuh", "ttt_internal.h"),
+    "ttt_mlp_tc_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
+    "ttt_mlp_generic_kernel": ("ttt_mlp_generic.cu", "common.cuh", "ttt_internal.h"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the source files a kernel is built from (its recorded counters
+    stay valid while this does not change)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "test_sequence_layers_ttt_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -99,7 +109,7 @@ def recorded_traffic(kernel: str, workload: str):
         for line in fh:
             f = line.split()
             if len(f) == 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
-                return int(f[3]) if f[2] == kernel_source_hash() else None
+                return int(f[3]) if f[2] == kernel_source_hash(kernel) else None
     return None
 
 
