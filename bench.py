@@ -83,6 +83,7 @@ KERNEL_SOURCES = {
     "ttt_linear_lag_kernel": ("ttt_linear_lag.cu", "ptx.cuh", "common.cuh", "tma_host.h", "ttt_internal.h"),
     "ttt_linear_generic_kernel": ("ttt_linear_generic.cu", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_tc_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
+    "ttt_mlp_split_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_generic_kernel": ("ttt_mlp_generic.cu", "common.cuh", "ttt_internal.h"),
 }
 
@@ -360,7 +361,8 @@ def run_ours(args, world, rank, local):
         if w.kind == "mlp":
             family = args.kernel if args.kernel != "auto" else ttt.mlp_pick_impl(
                 w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype)
-            kname = {"tensorcore": "ttt_mlp_tc_kernel", "generic": "ttt_mlp_generic_kernel"}[family]
+            kname = {"tensorcore": "ttt_mlp_tc_kernel", "tensorcore_split": "ttt_mlp_split_kernel",
+                     "generic": "ttt_mlp_generic_kernel"}[family]
             achieved, peak, bound, unit = af / (kernel_ms * 1e-3) / 1e12, bf16_tf, "tensor", "TFLOP/s"
         else:
             family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
@@ -397,7 +399,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
                     choices=[k for k, v in WORKLOADS.items() if v.T >= 2048])
-    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split"], default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,
                     help="CPU seconds of oracle work per reference sample")

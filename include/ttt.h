@@ -94,8 +94,11 @@ typedef enum { TTT_LN_RESIDUAL = 0, TTT_PLAIN = 1 } ttt_mode;
 typedef enum {
     TTT_IMPL_AUTO = 0,
     TTT_IMPL_GENERIC = 1,    /* fp32 SIMT scan: every supported shape, dtype and mode */
-    TTT_IMPL_TENSORCORE = 2  /* tensor-core scan: bf16 Q/K/V, b = 16, T a multiple of 16;
+    TTT_IMPL_TENSORCORE = 2, /* tensor-core scan: bf16 Q/K/V, b = 16, T a multiple of 16;
                                 TTT-Linear d = 64 in LN mode, TTT-MLP d = 64, hidden = 256 */
+    TTT_IMPL_TENSORCORE_SPLIT = 3 /* TTT-MLP only, same shapes as TTT_IMPL_TENSORCORE: each
+                                     scan's hidden units split over the two CTAs of a
+                                     cluster (two SMs per scan) */
 } ttt_impl;
 
 /*
@@ -148,10 +151,10 @@ ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batc
                            float* b1_T, float* W2_T, float* b2_T, ttt_stream_t stream);
 
 /* As ttt_mlp_forward, with an explicit kernel family (TTT_ERR_UNSUPPORTED if
- * that family does not cover the arguments).  The tensor-core family keeps the
- * state in shared memory in fp32 and runs every product on the tensor cores
- * (bf16 hi/lo operands, fp32 accumulation); its results agree with the generic
- * family's up to rounding. */
+ * that family does not cover the arguments).  The tensor-core families keep the
+ * state in shared memory in fp32 and run every product on the tensor cores
+ * (bf16 hi/lo operands, fp32 accumulation); their results agree with the
+ * generic family's, and with each other's, up to rounding. */
 ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                                 ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
                                 const void* V, const float* eta, const float* W1_0,
@@ -161,7 +164,10 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
                                 ttt_stream_t stream);
 
 /* Kernel family TTT_IMPL_AUTO would run for these TTT-MLP arguments
- * (TTT_IMPL_AUTO if no family covers them).  Pure host query. */
+ * (TTT_IMPL_AUTO if no family covers them).  Pure host query.  Among the
+ * tensor-core families it picks TTT_IMPL_TENSORCORE_SPLIT while the doubled
+ * grid, 2 B H CTAs of one SM each, fits in one wave (B H <= 74), else
+ * TTT_IMPL_TENSORCORE. */
 ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                            ttt_dtype qkv_dtype);
 

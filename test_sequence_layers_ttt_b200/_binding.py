@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
 
 TTT_BF16, TTT_F32 = 0, 1
 TTT_LN_RESIDUAL, TTT_PLAIN = 0, 1
-IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2}
+IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3}
+_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split"}
 STATUS = ["TTT_OK", "TTT_ERR_NULL", "TTT_ERR_SHAPE", "TTT_ERR_DTYPE", "TTT_ERR_ALIGN",
           "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT"]
 
@@ -63,14 +64,14 @@ def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
     code = lib.ttt_linear_pick_impl(B, H, T, d, mini_batch,
                                     TTT_BF16 if qkv_dtype in ("bf16", torch.bfloat16) else TTT_F32,
                                     _mode_code(mode))
-    return {0: "none", 1: "generic", 2: "tensorcore"}[code]
+    return _IMPL_NAMES[code]
 
 
 def mlp_pick_impl(B, H, T, d, hidden, mini_batch, qkv_dtype) -> str:
     """Kernel family the library's AUTO dispatch runs for these TTT-MLP arguments."""
     code = lib.ttt_mlp_pick_impl(B, H, T, d, hidden, mini_batch,
                                  TTT_BF16 if qkv_dtype in ("bf16", torch.bfloat16) else TTT_F32)
-    return {0: "none", 1: "generic", 2: "tensorcore"}[code]
+    return _IMPL_NAMES[code]
 
 
 def status_string(status: int) -> str:

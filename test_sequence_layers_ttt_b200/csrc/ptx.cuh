@@ -1,5 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA (bulk tensor) loads,
-// ldmatrix / movmatrix, mma.sync (bf16 -> fp32) and named barriers.
+// ldmatrix / movmatrix, mma.sync (bf16 -> fp32), named barriers, cluster
+// barriers and stores into a peer CTA's shared memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -91,6 +92,36 @@ __device__ __forceinline__ float bf16_hi_f32(uint32_t v) { return __uint_as_floa
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared-memory byte in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(local_addr), "r"(rank));
+    return d;
+}
+// Hardware cluster barrier, split in its two halves.  Every thread of every CTA
+// of the cluster arrives once per phase; arrive releases this thread's earlier
+// shared-memory writes (local and remote) at cluster scope, wait acquires them.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// plain stores into another CTA's shared memory (address from mapa_shared)
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float x, float y) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
 // ---------------------------------------------------------------- bf16 hi/lo split

@@ -153,6 +153,13 @@ ttt_status ttt_linear_forward(int B, int H, int T, int d, int mini_batch, ttt_dt
                                    W0, b0, ln_gamma, ln_beta, Z, W_T, b_T, TTT_IMPL_AUTO, stream);
 }
 
+// The family TTT_IMPL_AUTO runs for valid TTT-MLP arguments (TTT_IMPL_AUTO if none covers them)
+static ttt_impl mlp_auto_impl(const MlpArgs& a) {
+    if (ttt::mlp_split_supports(a) && (long)a.B * a.H <= ttt::kMlpSplitMaxScans) return TTT_IMPL_TENSORCORE_SPLIT;
+    if (ttt::mlp_tc_supports(a)) return TTT_IMPL_TENSORCORE;
+    return ttt::mlp_generic_supports(a) ? TTT_IMPL_GENERIC : TTT_IMPL_AUTO;
+}
+
 ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                                 ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
                                 const void* V, const float* eta, const float* W1_0, const float* b1_0,
@@ -164,15 +171,16 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
     ttt_status st = validate_mlp(a);
     if (st != TTT_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (impl == TTT_IMPL_AUTO) impl = mlp_auto_impl(a);
     switch (impl) {
-        case TTT_IMPL_AUTO:
-            if (ttt::mlp_tc_supports(a)) return finish(ttt::launch_mlp_tc(a, s), s);
-            return finish(ttt::launch_mlp_generic(a, s), s);
         case TTT_IMPL_GENERIC:
             return finish(ttt::launch_mlp_generic(a, s), s);
         case TTT_IMPL_TENSORCORE:
             if (!ttt::mlp_tc_supports(a)) return TTT_ERR_UNSUPPORTED;
             return finish(ttt::launch_mlp_tc(a, s), s);
+        case TTT_IMPL_TENSORCORE_SPLIT:
+            if (!ttt::mlp_split_supports(a)) return TTT_ERR_UNSUPPORTED;
+            return finish(ttt::launch_mlp_split(a, s), s);
         default:
             return TTT_ERR_UNSUPPORTED;
     }
@@ -182,8 +190,7 @@ ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batc
     MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, 1e-6f, nullptr, nullptr, nullptr, nullptr,
               nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
               nullptr};
-    if (ttt::mlp_tc_supports(a)) return TTT_IMPL_TENSORCORE;
-    return ttt::mlp_generic_supports(a) ? TTT_IMPL_GENERIC : TTT_IMPL_AUTO;
+    return mlp_auto_impl(a);
 }
 
 ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batch,

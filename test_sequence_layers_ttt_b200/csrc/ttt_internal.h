@@ -38,6 +38,13 @@ cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);
 bool mlp_tc_supports(const MlpArgs& a);
 cudaError_t launch_mlp_tc(const MlpArgs& a, cudaStream_t stream);
 
+// Hidden units of each scan split over a 2-CTA cluster; same shapes as mlp_tc.
+// Preferred while its 2 B H CTAs (one per SM) fit in one wave: a 148-SM B200
+// holds 74 such clusters at once (cudaOccupancyMaxActiveClusters).
+constexpr int kMlpSplitMaxScans = 74;
+bool mlp_split_supports(const MlpArgs& a);
+cudaError_t launch_mlp_split(const MlpArgs& a, cudaStream_t stream);
+
 // Device-side error word set by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_device_error(unsigned int* out);
 

@@ -545,6 +545,499 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
     if (tid < D) b2_T[bh * D + tid] = s.b2[tid];
 }
 
+// ============================================================================
+// Split variant: the hidden units of one scan are divided between the two CTAs
+// of a cluster (CTA r owns units [128r, 128r + 128) of W1's columns, b1, and
+// W2's rows); both hold the full b2, gamma, beta and the chunk's tokens.  Every
+// product over the hidden units is formed as two partial sums that the CTAs
+// swap through distributed shared memory; the rest is either local to a
+// hidden slice or repeated bit for bit in both CTAs:
+//   Z1, H, G1, Z1q, Hq, the W1 / b1 / W2 updates   local to the slice
+//   Y  = b2 + H_0 W2_0 + H_1 W2_1                   partial sums swapped
+//   G2, E2 = -eta G2, A, the b2 update              repeated in both CTAs
+//   Hq H^T and Hq W2                                partial sums swapped
+// Both CTAs add the partials in rank order, so their copies of Y, G2, b2 and
+// Z2q agree exactly.  CTA r writes the outputs of tokens [8r, 8r + 8) of each
+// chunk.  Two hardware cluster barriers per chunk order the swaps; the W1 and
+// W2 updates run between the arrive and the wait of the second one.
+namespace split {
+
+constexpr int kSplit = 2;
+constexpr int HL = HID / kSplit;  // hidden units per CTA
+constexpr int NPL = HL / 64;      // 64-column panels of a [16][HL] activation
+
+// W2^T slice [out][HL], rows XOR-swizzled in 8-float groups
+__device__ __forceinline__ int w2i(int out, int hid) { return out * HL + ((((hid >> 3) ^ (out & 7))) << 3) + (hid & 7); }
+
+struct Smem {
+    float w1t[HL * D];  // W1^T slice [hid][in], swizzled with w1i
+    float w2t[D * HL];  // W2^T slice [out][hid], swizzled with w2i
+    float b1[HL], b2[D];
+    float gam[D], bet[D];
+    unsigned char K[PANEL], V[PANEL], Q[PANEL];
+    unsigned char Hh[NPL][PANEL], Hl[NPL][PANEL];
+    unsigned char Hqh[NPL][PANEL], Hql[NPL][PANEL];
+    unsigned char G1h[NPL][PANEL], G1l[NPL][PANEL];
+    unsigned char G2h[PANEL], G2l[PANEL];
+    unsigned char E2h[PANEL], E2l[PANEL];
+    unsigned char EXh[PANEL], EXl[PANEL];
+    float yp[kSplit][kChunk * YLD];  // H W2 partial of CTA r (written by CTA r in both CTAs)
+    float zp[kSplit][kChunk * YLD];  // Hq W2 partial of CTA r
+    float Y[kChunk * YLD];           // Z2q
+    uint4 afrag[2][32];
+    float4 a2p[kSplit * NPL][2][32];  // Hq H^T partial of CTA r, panel p at [NPL r + p]
+    alignas(16) float eta[kChunk];
+};
+
+// d_h += ah bh, d_l += ah bl + al bh: the split product in two accumulators
+__device__ __forceinline__ void mma3s(float (&dh)[4], float (&dl)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
+                                      uint32_t bh0, uint32_t bh1, uint32_t bl0, uint32_t bl1) {
+    mma(dh, ah, bh0, bh1);
+    mma(dl, ah, bl0, bl1);
+    mma(dl, al, bh0, bh1);
+}
+
+}  // namespace split
+
+__global__ void __cluster_dims__(split::kSplit, 1, 1) __launch_bounds__(kThreads, 1)
+ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ Kg,
+                     const __nv_bfloat16* __restrict__ Vg, const float* __restrict__ etag, const float* W1_0,
+                     const float* b1_0, const float* W2_0, const float* b2_0, const float* __restrict__ gamma,
+                     const float* __restrict__ beta, float* __restrict__ Z, float* W1_T, float* b1_T, float* W2_T,
+                     float* b2_T) {
+    using split::HL;
+    using split::NPL;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    split::Smem& s = *reinterpret_cast<split::Smem*>(smem_raw + ((128u - (ptx::smem_addr(smem_raw) & 127u)) & 127u));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t rank = ptx::cluster_ctarank(), peer = rank ^ 1u;
+    const long bh = blockIdx.x / split::kSplit;
+    const int h = (int)(bh % H);
+    const int n = T / kChunk;
+    const int hid0 = HL * (int)rank;  // first hidden unit of this CTA's slice
+    auto remote = [&](const void* p) { return ptx::mapa_shared(ptx::smem_addr(p), peer); };
+
+    // ---- initial state: this CTA's slice of W1, b1, W2; all of b2
+    for (int i = tid; i < D * HL; i += kThreads) {
+        const int in = i / HL, hl = i % HL;  // W1_0 [in][hid]
+        s.w1t[w1i(hl, in)] = W1_0[bh * D * HID + (long)in * HID + hid0 + hl];
+    }
+    for (int i = tid; i < HL * D; i += kThreads) {
+        const int hl = i / D, out = i % D;  // W2_0 [hid][out]
+        s.w2t[split::w2i(out, hl)] = W2_0[bh * HID * D + (long)(hid0 + hl) * D + out];
+    }
+    for (int i = tid; i < HL; i += kThreads) s.b1[i] = b1_0[bh * HID + hid0 + i];
+    if (tid < D) {
+        s.b2[tid] = b2_0[bh * D + tid];
+        s.gam[tid] = gamma[(long)h * D + tid];
+        s.bet[tid] = beta[(long)h * D + tid];
+    }
+
+    // ---- token loads (both CTAs read the whole chunk): as in the one-CTA kernel
+    const long tok0 = bh * (long)T;
+    const int lt = tid >> 7, lidx = tid & 127, lrow = lidx >> 3, lchunk = lidx & 7;
+    const __nv_bfloat16* lsrc = lt == 0 ? Kg : (lt == 1 ? Vg : Qg);
+    uint4 pf = make_uint4(0u, 0u, 0u, 0u);
+    float4 pfe = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fetch = [&](int c) {
+        if (tid < 384) pf = *reinterpret_cast<const uint4*>(lsrc + (tok0 + c * kChunk + lrow) * D + lchunk * 8);
+        else if (tid < 388) pfe = *reinterpret_cast<const float4*>(etag + tok0 + c * kChunk + (tid - 384) * 4);
+    };
+    if (n > 0) fetch(0);
+
+    const uint32_t sK = ptx::smem_addr(s.K), sQ = ptx::smem_addr(s.Q);
+    float* Zbh = Z + tok0 * D;
+    // this warp's hidden units [8 warp, 8 warp + 8): panel and column inside it
+    const int p = warp >> 3, pc = 8 * (warp & 7) + 2 * t;
+
+    // the peer CTA is running before any store reaches its shared memory
+    ptx::cluster_arrive();
+    ptx::cluster_wait();
+
+    for (int c = 0; c < n; c++) {
+        // ================================================= phase 0: this chunk's tokens in, next chunk's requested
+        __syncthreads();
+        if (tid < 384) {
+            unsigned char* dst = lt == 0 ? s.K : (lt == 1 ? s.V : s.Q);
+            *reinterpret_cast<uint4*>(dst + swz_chunk(lrow, lchunk)) = pf;
+        } else if (tid < 388) {
+            *reinterpret_cast<float4*>(&s.eta[(tid - 384) * 4]) = pfe;
+        }
+        if (c + 1 < n) fetch(c + 1);
+        __syncthreads();
+
+        // ================================================= phase 1: [X; Q] W1 + b1 on this warp's 8 hidden units, H = GELU(Z1)
+        float z1[4], zq[4], sg1[4];
+        {
+            float z1l[4], zql[4];
+            zero(z1l);
+            zero(zql);
+            const int col = 8 * warp + 2 * t;
+            z1[0] = z1[2] = zq[0] = zq[2] = s.b1[col];
+            z1[1] = z1[3] = zq[1] = zq[3] = s.b1[col + 1];
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++) {
+                uint32_t ax[4], aq[4];
+                ld_a(sK, ks, lane, ax);
+                ld_a(sQ, ks, lane, aq);
+                const int hid = 8 * warp + g, in = 16 * ks + 2 * t;
+                const float2 w0 = *reinterpret_cast<const float2*>(&s.w1t[w1i(hid, in)]);
+                const float2 w1 = *reinterpret_cast<const float2*>(&s.w1t[w1i(hid, in + 8)]);
+                uint32_t bh0, bl0, bh1, bl1;
+                ptx::split_pair(w0.x, w0.y, bh0, bl0);
+                ptx::split_pair(w1.x, w1.y, bh1, bl1);
+                mma(z1, ax, bh0, bh1);
+                mma(z1l, ax, bl0, bl1);
+                mma(zq, aq, bh0, bh1);
+                mma(zql, aq, bl0, bl1);
+            }
+            float hv[4];
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                z1[r] += z1l[r];
+                zq[r] += zql[r];
+                hv[r] = gelu_sig(z1[r], sg1[r]);
+            }
+            store_pairs(s.Hh[p], s.Hl[p], g, pc, hv);
+        }
+        __syncthreads();
+
+        // ================================================= phase 2: partial Y = H W2 (warps 0-7), A and -eta X (warps 8-15)
+        if (warp < 8) {
+            float acc[4], accl[4], acc2[4], acc2l[4];
+            zero(acc);
+            zero(accl);
+            zero(acc2);
+            zero(acc2l);
+#pragma unroll 4
+            for (int ks = 0; ks < 4 * NPL; ks++) {
+                uint32_t ah[4], al[4];
+                ld_a(ptx::smem_addr(s.Hh[ks >> 2]), ks & 3, lane, ah);
+                ld_a(ptx::smem_addr(s.Hl[ks >> 2]), ks & 3, lane, al);
+                const int out = 8 * warp + g, hid = 16 * ks + 2 * t;
+                const float2 w0 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid)]);
+                const float2 w1 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid + 8)]);
+                uint32_t bh0, bl0, bh1, bl1;
+                ptx::split_pair(w0.x, w0.y, bh0, bl0);
+                ptx::split_pair(w1.x, w1.y, bh1, bl1);
+                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, bh0, bh1, bl0, bl1);
+                else split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) + (acc2[r] + acc2l[r]);
+            const int col = 8 * warp + 2 * t;
+            float* y0 = &s.yp[rank][g * YLD + col];
+            float* y1 = &s.yp[rank][(g + 8) * YLD + col];
+            *reinterpret_cast<float2*>(y0) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2*>(y1) = make_float2(acc[2], acc[3]);
+            ptx::st_cluster_f32x2(remote(y0), acc[0], acc[1]);
+            ptx::st_cluster_f32x2(remote(y1), acc[2], acc[3]);
+        } else {
+            if (warp == 8) {
+                // A = tril(eta_s (q_t . x_s + 1)) as -A hi/lo A fragments
+                float pa[2][4];
+                zero(pa[0]);
+                zero(pa[1]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ks++) {
+                    uint32_t aq[4], bx[4];
+                    ld_a(sQ, ks, lane, aq);
+                    ld_b_col(sK, ks, lane, bx);
+                    mma(pa[0], aq, bx[0], bx[1]);
+                    mma(pa[1], aq, bx[2], bx[3]);
+                }
+                uint4 hi, lo;
+                causal_frag(pa, s.eta, g, t, hi, lo);
+                s.afrag[0][lane] = hi;
+                s.afrag[1][lane] = lo;
+            }
+            // -eta_t X[t][:] for the W1 update (k = tokens): 256 threads, two pairs each
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const int i = tid - 256 + 256 * k, row = i >> 5, col = 2 * (i & 31);
+                const uint32_t xv = *reinterpret_cast<const uint32_t*>(s.K + swz(row, col));
+                const float e = -s.eta[row];
+                uint32_t hi, lo;
+                ptx::split_pair(e * ptx::bf16_lo_f32(xv), e * ptx::bf16_hi_f32(xv), hi, lo);
+                *reinterpret_cast<uint32_t*>(s.EXh + swz(row, col)) = hi;
+                *reinterpret_cast<uint32_t*>(s.EXl + swz(row, col)) = lo;
+            }
+        }
+        ptx::cluster_arrive();
+        ptx::cluster_wait();
+
+        // ================================================= phase 3: Y = b2 + partials, G2 = dl/dY, E2 = -eta G2 (warp w: token w)
+        {
+            const int row = warp, col = 2 * lane;
+            const float2 p0 = *reinterpret_cast<const float2*>(&s.yp[0][row * YLD + col]);
+            const float2 p1 = *reinterpret_cast<const float2*>(&s.yp[1][row * YLD + col]);
+            const float y0 = s.b2[col] + p0.x + p1.x, y1 = s.b2[col + 1] + p0.y + p1.y;
+            const uint32_t xv = *reinterpret_cast<const uint32_t*>(s.K + swz(row, col));
+            const uint32_t vv = *reinterpret_cast<const uint32_t*>(s.V + swz(row, col));
+            const float mu = warp_sum(y0 + y1) * (1.f / D);
+            const float d0 = y0 - mu, d1 = y1 - mu;
+            const float rs = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / D) + eps);
+            const float xh0 = d0 * rs, xh1 = d1 * rs;
+            const float g0 = s.gam[col], g1 = s.gam[col + 1];
+            const float gx0 = 2.f * g0 * (ptx::bf16_lo_f32(xv) + g0 * xh0 + s.bet[col] - ptx::bf16_lo_f32(vv));
+            const float gx1 = 2.f * g1 * (ptx::bf16_hi_f32(xv) + g1 * xh1 + s.bet[col + 1] - ptx::bf16_hi_f32(vv));
+            const float mgx = warp_sum(gx0 + gx1) * (1.f / D);
+            const float mgxx = warp_sum(gx0 * xh0 + gx1 * xh1) * (1.f / D);
+            const float G0 = rs * (gx0 - mgx - xh0 * mgxx), G1 = rs * (gx1 - mgx - xh1 * mgxx);
+            const float e = -s.eta[row];
+            uint32_t hi, lo;
+            ptx::split_pair(G0, G1, hi, lo);
+            *reinterpret_cast<uint32_t*>(s.G2h + swz(row, col)) = hi;
+            *reinterpret_cast<uint32_t*>(s.G2l + swz(row, col)) = lo;
+            ptx::split_pair(e * G0, e * G1, hi, lo);
+            *reinterpret_cast<uint32_t*>(s.E2h + swz(row, col)) = hi;
+            *reinterpret_cast<uint32_t*>(s.E2l + swz(row, col)) = lo;
+        }
+        __syncthreads();
+
+        // ================================================= phase 4: G1 = (G2 W2^T) * GELU'(Z1) on this warp's hidden units
+        {
+            float acc[4], accl[4];
+            zero(acc);
+            zero(accl);
+            const uint32_t g2h = ptx::smem_addr(s.G2h), g2l = ptx::smem_addr(s.G2l);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++) {
+                uint32_t ah[4], al[4];
+                ld_a(g2h, ks, lane, ah);
+                ld_a(g2l, ks, lane, al);
+                const int hid = 8 * warp + g, out = 16 * ks + 2 * t;
+                uint32_t bh0, bl0, bh1, bl1;
+                ptx::split_pair(s.w2t[split::w2i(out, hid)], s.w2t[split::w2i(out + 1, hid)], bh0, bl0);
+                ptx::split_pair(s.w2t[split::w2i(out + 8, hid)], s.w2t[split::w2i(out + 9, hid)], bh1, bl1);
+                split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) * gelu_prime_sig(z1[r], sg1[r]);
+            store_pairs(s.G1h[p], s.G1l[p], g, pc, acc);
+        }
+        __syncthreads();
+
+        // ================================================= phase 5: Z1q = Q W1 + b1 - A G1, Hq = GELU(Z1q)
+        {
+            const uint4 fh = s.afrag[0][lane], fl = s.afrag[1][lane];
+            const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
+            uint32_t bh[4], bl[4];
+            ld_b_tok(ptx::smem_addr(s.G1h[p]), (warp & 7) >> 1, lane, bh);
+            ld_b_tok(ptx::smem_addr(s.G1l[p]), (warp & 7) >> 1, lane, bl);
+            const int o = 2 * (warp & 1);
+            mma3(zq, ah, al, bh[o], bh[o + 1], bl[o], bl[o + 1]);
+            float hv[4], sq;
+#pragma unroll
+            for (int r = 0; r < 4; r++) hv[r] = gelu_sig(zq[r], sq);
+            store_pairs(s.Hqh[p], s.Hql[p], g, pc, hv);
+        }
+        __syncthreads();
+
+        // ================================================= phase 6: partial Hq H^T (warps 0-1), partial Hq W2 (warps 8-15);
+        // then, between the arrive and the wait, the W1 / b1 (warps 0-7) and W2 (warps 8-15) updates
+        if (warp < NPL) {
+            const int pp = warp;
+            float acc[2][4];
+            zero(acc[0]);
+            zero(acc[1]);
+#pragma unroll
+            for (int kb = 0; kb < 4; kb++) {
+                uint32_t ah[4], al[4], bh[4], bl[4];
+                ld_a(ptx::smem_addr(s.Hqh[pp]), kb, lane, ah);
+                ld_a(ptx::smem_addr(s.Hql[pp]), kb, lane, al);
+                ld_b_col(ptx::smem_addr(s.Hh[pp]), kb, lane, bh);
+                ld_b_col(ptx::smem_addr(s.Hl[pp]), kb, lane, bl);
+                mma3(acc[0], ah, al, bh[0], bh[1], bl[0], bl[1]);
+                mma3(acc[1], ah, al, bh[2], bh[3], bl[2], bl[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; nt++) {
+                float4* dst = &s.a2p[NPL * rank + pp][nt][lane];
+                const float4 v = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+                *dst = v;
+                ptx::st_cluster_f32x4(remote(dst), v);
+            }
+        } else if (warp >= 8) {
+            const int ot = warp - 8;  // output columns [8 ot, 8 ot + 8)
+            float acc[4], accl[4], acc2[4], acc2l[4];
+            zero(acc);
+            zero(accl);
+            zero(acc2);
+            zero(acc2l);
+#pragma unroll 4
+            for (int ks = 0; ks < 4 * NPL; ks++) {
+                uint32_t ah[4], al[4];
+                ld_a(ptx::smem_addr(s.Hqh[ks >> 2]), ks & 3, lane, ah);
+                ld_a(ptx::smem_addr(s.Hql[ks >> 2]), ks & 3, lane, al);
+                const int out = 8 * ot + g, hid = 16 * ks + 2 * t;
+                const float2 w0 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid)]);
+                const float2 w1 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid + 8)]);
+                uint32_t bh0, bl0, bh1, bl1;
+                ptx::split_pair(w0.x, w0.y, bh0, bl0);
+                ptx::split_pair(w1.x, w1.y, bh1, bl1);
+                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, bh0, bh1, bl0, bl1);
+                else split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) + (acc2[r] + acc2l[r]);
+            const int col = 8 * ot + 2 * t;
+            float* z0 = &s.zp[rank][g * YLD + col];
+            float* z1p = &s.zp[rank][(g + 8) * YLD + col];
+            *reinterpret_cast<float2*>(z0) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2*>(z1p) = make_float2(acc[2], acc[3]);
+            ptx::st_cluster_f32x2(remote(z0), acc[0], acc[1]);
+            ptx::st_cluster_f32x2(remote(z1p), acc[2], acc[3]);
+            // every read of W2 in this chunk is done before any warp updates it
+            ptx::named_bar_sync(2, 256);
+        }
+        ptx::cluster_arrive();
+        if (warp < 8) {
+            // W1^T[hid][in] += G1^T (-eta X), b1 += G1^T (-eta); hidden rows [16 warp, 16 warp + 16)
+            uint32_t eh[2], el[2];  // -eta as a B column (n = 0): k = tokens 2t..2t+1 and 2t+8..2t+9
+            ptx::split_pair(g == 0 ? -s.eta[2 * t] : 0.f, g == 0 ? -s.eta[2 * t + 1] : 0.f, eh[0], el[0]);
+            ptx::split_pair(g == 0 ? -s.eta[2 * t + 8] : 0.f, g == 0 ? -s.eta[2 * t + 9] : 0.f, eh[1], el[1]);
+            const int mt = warp, p1 = mt >> 2;
+            uint32_t ah[4], al[4];
+            ld_a_t(ptx::smem_addr(s.G1h[p1]), mt & 3, lane, ah);
+            ld_a_t(ptx::smem_addr(s.G1l[p1]), mt & 3, lane, al);
+#pragma unroll
+            for (int jp = 0; jp < 4; jp++) {
+                uint32_t bh[4], bl[4];
+                ld_b_tok(ptx::smem_addr(s.EXh), jp, lane, bh);
+                ld_b_tok(ptx::smem_addr(s.EXl), jp, lane, bl);
+                float d[2][4];
+                zero(d[0]);
+                zero(d[1]);
+                mma3(d[0], ah, al, bh[0], bh[1], bl[0], bl[1]);
+                mma3(d[1], ah, al, bh[2], bh[3], bl[2], bl[3]);
+#pragma unroll
+                for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                    for (int rh = 0; rh < 2; rh++) {
+                        float2* wp = reinterpret_cast<float2*>(&s.w1t[w1i(16 * mt + g + 8 * rh, 16 * jp + 8 * nt + 2 * t)]);
+                        float2 wv = *wp;
+                        wv.x += d[nt][2 * rh];
+                        wv.y += d[nt][2 * rh + 1];
+                        *wp = wv;
+                    }
+            }
+            float db[4];
+            zero(db);
+            mma3(db, ah, al, eh[0], eh[1], el[0], el[1]);
+            if (t == 0) {
+                s.b1[16 * mt + g] += db[0];
+                s.b1[16 * mt + 8 + g] += db[2];
+            }
+        } else {
+            // W2^T[out][hid] += E2^T H; output rows [16 mo, 16 mo + 16), hidden panel pp
+            const int v = warp - 8, mo = v & 3, pp = v >> 2;
+            uint32_t ah[4], al[4];
+            ld_a_t(ptx::smem_addr(s.E2h), mo, lane, ah);
+            ld_a_t(ptx::smem_addr(s.E2l), mo, lane, al);
+#pragma unroll
+            for (int jp = 0; jp < 4; jp++) {
+                uint32_t bh[4], bl[4];
+                ld_b_tok(ptx::smem_addr(s.Hh[pp]), jp, lane, bh);
+                ld_b_tok(ptx::smem_addr(s.Hl[pp]), jp, lane, bl);
+                float d[2][4];
+                zero(d[0]);
+                zero(d[1]);
+                mma3(d[0], ah, al, bh[0], bh[1], bl[0], bl[1]);
+                mma3(d[1], ah, al, bh[2], bh[3], bl[2], bl[3]);
+#pragma unroll
+                for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                    for (int rh = 0; rh < 2; rh++) {
+                        float2* wp = reinterpret_cast<float2*>(
+                            &s.w2t[split::w2i(16 * mo + g + 8 * rh, 64 * pp + 16 * jp + 8 * nt + 2 * t)]);
+                        float2 wv = *wp;
+                        wv.x += d[nt][2 * rh];
+                        wv.y += d[nt][2 * rh + 1];
+                        *wp = wv;
+                    }
+            }
+        }
+        ptx::cluster_wait();
+
+        // ================================================= phase 7 (warps 0-7): Z2q = b2 + partials - A2 G2, b2 update,
+        // z = q + LN(Z2q) for this CTA's 8 tokens
+        if (warp < 8) {
+            const int v = warp;  // output columns [8v, 8v + 8)
+            float pa[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; nt++) {
+                float4 a = s.a2p[0][nt][lane];
+#pragma unroll
+                for (int q = 1; q < split::kSplit * NPL; q++) {
+                    const float4 b = s.a2p[q][nt][lane];
+                    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+                }
+                pa[nt][0] = a.x; pa[nt][1] = a.y; pa[nt][2] = a.z; pa[nt][3] = a.w;
+            }
+            uint4 fh, fl;
+            causal_frag(pa, s.eta, g, t, fh, fl);
+            const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
+            const int col = 8 * v + 2 * t;
+            const float2 p00 = *reinterpret_cast<const float2*>(&s.zp[0][g * YLD + col]);
+            const float2 p10 = *reinterpret_cast<const float2*>(&s.zp[1][g * YLD + col]);
+            const float2 p01 = *reinterpret_cast<const float2*>(&s.zp[0][(g + 8) * YLD + col]);
+            const float2 p11 = *reinterpret_cast<const float2*>(&s.zp[1][(g + 8) * YLD + col]);
+            const float bb0 = s.b2[col], bb1 = s.b2[col + 1];
+            float z2[4] = {bb0 + p00.x + p10.x, bb1 + p00.y + p10.y, bb0 + p01.x + p11.x, bb1 + p01.y + p11.y};
+            uint32_t bh[4], bl[4];
+            ld_b_tok(ptx::smem_addr(s.G2h), v >> 1, lane, bh);
+            ld_b_tok(ptx::smem_addr(s.G2l), v >> 1, lane, bl);
+            const int o = (v & 1) * 2;
+            mma3(z2, ah, al, bh[o], bh[o + 1], bl[o], bl[o + 1]);
+            *reinterpret_cast<float2*>(&s.Y[g * YLD + col]) = make_float2(z2[0], z2[1]);
+            *reinterpret_cast<float2*>(&s.Y[(g + 8) * YLD + col]) = make_float2(z2[2], z2[3]);
+            // every read of b2 and of Z2q's producers in this chunk is done
+            ptx::named_bar_sync(1, 256);
+            if (v < 4) {
+                // b2 += E2^T 1 for output rows [16v, 16v + 16)
+                uint32_t eh4[4], el4[4];
+                ld_a_t(ptx::smem_addr(s.E2h), v, lane, eh4);
+                ld_a_t(ptx::smem_addr(s.E2l), v, lane, el4);
+                const uint32_t ones = g == 0 ? 0x3f803f80u : 0u;  // (1, 1) in bf16 on column 0
+                float db[4];
+                zero(db);
+                mma(db, eh4, ones, ones);
+                mma(db, el4, ones, ones);
+                if (t == 0) {
+                    s.b2[16 * v + g] += db[0];
+                    s.b2[16 * v + 8 + g] += db[2];
+                }
+            }
+            {
+                const int row = 8 * (int)rank + v, cc = 2 * lane;
+                const float2 zz = *reinterpret_cast<const float2*>(&s.Y[row * YLD + cc]);
+                const float mu = warp_sum(zz.x + zz.y) * (1.f / D);
+                const float d0 = zz.x - mu, d1 = zz.y - mu;
+                const float rs = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / D) + eps);
+                const uint32_t qv = *reinterpret_cast<const uint32_t*>(s.Q + swz(row, cc));
+                float2 o2;
+                o2.x = ptx::bf16_lo_f32(qv) + s.gam[cc] * d0 * rs + s.bet[cc];
+                o2.y = ptx::bf16_hi_f32(qv) + s.gam[cc + 1] * d1 * rs + s.bet[cc + 1];
+                *reinterpret_cast<float2*>(Zbh + (size_t)(c * kChunk + row) * D + cc) = o2;
+            }
+        }
+    }
+    __syncthreads();
+    // ---- final state: this CTA's slice; CTA 0 writes b2
+    for (int i = tid; i < D * HL; i += kThreads) {
+        const int in = i / HL, hl = i % HL;
+        W1_T[bh * D * HID + (long)in * HID + hid0 + hl] = s.w1t[w1i(hl, in)];
+    }
+    for (int i = tid; i < HL * D; i += kThreads) {
+        const int hl = i / D, out = i % D;
+        W2_T[bh * HID * D + (long)(hid0 + hl) * D + out] = s.w2t[split::w2i(out, hl)];
+    }
+    for (int i = tid; i < HL; i += kThreads) b1_T[bh * HID + hid0 + i] = s.b1[i];
+    if (rank == 0 && tid < D) b2_T[bh * D + tid] = s.b2[tid];
+}
+
 }  // namespace
 
 bool mlp_tc_supports(const MlpArgs& a) {
@@ -558,6 +1051,20 @@ cudaError_t launch_mlp_tc(const MlpArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(ttt_mlp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ttt_mlp_tc_kernel<<<a.B * a.H, kThreads, smem, stream>>>(
+        a.T, a.H, a.ln_eps, static_cast<const __nv_bfloat16*>(a.Q), static_cast<const __nv_bfloat16*>(a.K),
+        static_cast<const __nv_bfloat16*>(a.V), a.eta, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma, a.beta, a.Z,
+        a.W1_T, a.b1_T, a.W2_T, a.b2_T);
+    return cudaPeekAtLastError();
+}
+
+bool mlp_split_supports(const MlpArgs& a) { return mlp_tc_supports(a); }
+
+cudaError_t launch_mlp_split(const MlpArgs& a, cudaStream_t stream) {
+    if (!mlp_split_supports(a)) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(split::Smem) + 128;
+    cudaError_t e = cudaFuncSetAttribute(ttt_mlp_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ttt_mlp_split_kernel<<<a.B * a.H * split::kSplit, kThreads, smem, stream>>>(
         a.T, a.H, a.ln_eps, static_cast<const __nv_bfloat16*>(a.Q), static_cast<const __nv_bfloat16*>(a.K),
         static_cast<const __nv_bfloat16*>(a.V), a.eta, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma, a.beta, a.Z,
         a.W1_T, a.b1_T, a.W2_T, a.b2_T);

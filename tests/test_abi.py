@@ -139,6 +139,12 @@ def test_mlp_alias_and_align():
     assert mlp_call(ptrs=with_ptr(13, fake(13) + 4, 15)) == ALIGN
 
 
+def test_linear_has_no_split_family():
+    # the split family is TTT-MLP only; unknown families are refused before any launch
+    assert linear_call(impl=3) == UNSUP
+    assert linear_call(impl=9) == UNSUP
+
+
 def test_pick_impl_is_a_host_query():
     f = b.lib.ttt_linear_pick_impl
     assert f(1, 2, 64, 16, 16, 1, 0) == 1        # fp32 d=16: generic
@@ -157,7 +163,12 @@ def test_host_pipeline_groups_cover_every_scan_once(B, H, n):
 
 def test_mlp_pick_impl_is_a_host_query():
     from test_sequence_layers_ttt_b200 import _binding as ttt
-    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "bf16") == "tensorcore"
+    # two SMs per scan while 2 B H CTAs fit in one wave, one SM per scan beyond
+    assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "bf16") == "tensorcore_split"
+    assert ttt.mlp_pick_impl(4, 16, 8192, 64, 256, 16, "bf16") == "tensorcore_split"
+    assert ttt.mlp_pick_impl(2, 37, 8192, 64, 256, 16, "bf16") == "tensorcore_split"
+    assert ttt.mlp_pick_impl(5, 15, 8192, 64, 256, 16, "bf16") == "tensorcore"
+    assert ttt.mlp_pick_impl(8, 32, 2048, 64, 256, 16, "bf16") == "tensorcore"
     assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 16, "f32") == "generic"
     assert ttt.mlp_pick_impl(4, 12, 8192, 64, 256, 32, "bf16") == "generic"
     assert ttt.mlp_pick_impl(4, 12, 8200, 64, 256, 16, "bf16") == "generic"

@@ -266,6 +266,10 @@ def test_linear_host_pipeline_uneven_groups(ttt, mode):
 
 # ------------------------------------------------------------------ TTT-MLP
 
+# the tensor-core families: one CTA per scan, and each scan's hidden units
+# split over a 2-CTA cluster
+TC_MLP = ["tensorcore", "tensorcore_split"]
+
 def gpu_mlp(ttt, w, inp, mini_batch=None, impl="auto"):
     g = to_cuda(inp)
     out = ttt.ttt_mlp_forward(*(g[k] for k in MLP_KEYS), mini_batch=mini_batch or w.mini_batch,
@@ -310,19 +314,37 @@ def test_mlp_f32_inputs(ttt):
 
 
 def test_mlp_full_sampled_heads(ttt):
-    """The benchmarked launch (tensor-core family): all 48 scans of 8k tokens on
-    the GPU, three checked end to end against the oracle."""
+    """The benchmarked launch (the split tensor-core family): all 48 scans of 8k
+    tokens on the GPU, three checked end to end against the oracle."""
     w = WORKLOADS["mlp_8k"]
-    assert ttt.mlp_pick_impl(w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype) == "tensorcore"
+    assert ttt.mlp_pick_impl(w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype) == "tensorcore_split"
     compare_mlp(ttt, w, make_inputs(w, 0), pairs=[(0, 0), (2, 7), (3, 11)])
 
 
+@pytest.mark.parametrize("impl", TC_MLP)
 @pytest.mark.parametrize("T", [16, 48, 256, 1024])
 @pytest.mark.parametrize("seed", [0, 1])
-def test_mlp_tensorcore_vs_oracle(ttt, T, seed):
-    """Several chunks, all heads of a small batch, the tensor-core family explicitly."""
+def test_mlp_tensorcore_vs_oracle(ttt, T, seed, impl):
+    """Several chunks, all heads of a small batch, each tensor-core family explicitly."""
     w = WORKLOADS["mlp_8k"].with_shape(B=2, H=3, T=T)
-    compare_mlp(ttt, w, make_inputs(w, seed), impl="tensorcore")
+    compare_mlp(ttt, w, make_inputs(w, seed), impl=impl)
+
+
+def test_mlp_full_sampled_heads_one_cta_family(ttt):
+    """The one-CTA family on the full 8k workload, as AUTO runs it when 2 B H
+    CTAs no longer fit in one wave."""
+    w = WORKLOADS["mlp_8k"]
+    compare_mlp(ttt, w, make_inputs(w, 1), pairs=[(1, 3), (3, 0)], impl="tensorcore")
+
+
+def test_mlp_split_matches_one_cta_family(ttt):
+    """The two tensor-core families differ only in summation order."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=1024)
+    inp = make_inputs(w, 10)
+    a = gpu_mlp(ttt, w, inp, impl="tensorcore_split")
+    b = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    for name, x, y in zip(("Z", "W1_T", "b1_T", "W2_T", "b2_T"), a, b):
+        assert_close(x, y.astype(np.float64), 1e-4, f"{name} split vs one CTA", denom=max(rms(y), 1e-3))
 
 
 def test_mlp_generic_explicit_on_the_tensorcore_shape(ttt):
@@ -330,40 +352,43 @@ def test_mlp_generic_explicit_on_the_tensorcore_shape(ttt):
     compare_mlp(ttt, w, make_inputs(w, 4), impl="generic")
 
 
-def test_mlp_tensorcore_matches_generic(ttt):
+@pytest.mark.parametrize("impl", TC_MLP)
+def test_mlp_tensorcore_matches_generic(ttt, impl):
     w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=512)
     inp = make_inputs(w, 9)
-    tc = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    tc = gpu_mlp(ttt, w, inp, impl=impl)
     ge = gpu_mlp(ttt, w, inp, impl="generic")
     for name, a, b in zip(("Z", "W1_T", "b1_T", "W2_T", "b2_T"), tc, ge):
         assert_close(a, b.astype(np.float64), 1e-3, f"{name} tensorcore vs generic",
                      denom=max(rms(b), 1e-3))
 
 
-def test_mlp_tensorcore_continuation(ttt):
+@pytest.mark.parametrize("impl", TC_MLP)
+def test_mlp_tensorcore_continuation(ttt, impl):
     """Two calls split at a mini-batch boundary, the state carried through the
     final-state buffers, equal one call up to rounding."""
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=256)
     inp = make_inputs(w, 5)
-    full = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    full = gpu_mlp(ttt, w, inp, impl=impl)
     half = w.with_shape(T=128)
     first = {k: (v[:, :, :128].contiguous() if k in ("Q", "K", "V", "eta") else v) for k, v in inp.items()}
-    out1 = gpu_mlp(ttt, half, first, impl="tensorcore")
+    out1 = gpu_mlp(ttt, half, first, impl=impl)
     second = {k: (v[:, :, 128:].contiguous() if k in ("Q", "K", "V", "eta") else v) for k, v in inp.items()}
     for k, o in zip(("W1_0", "b1_0", "W2_0", "b2_0"), out1[1:]):
         second[k] = torch.from_numpy(o)
-    out2 = gpu_mlp(ttt, half, second, impl="tensorcore")
+    out2 = gpu_mlp(ttt, half, second, impl=impl)
     Z = np.concatenate([out1[0], out2[0]], axis=2)
     assert_close(Z, full[0].astype(np.float64), 1e-4, "Z continuation")
     for name, a, b in zip(("W1_T", "b1_T", "W2_T", "b2_T"), out2[1:], full[1:]):
         assert_close(a, b.astype(np.float64), 1e-4, name, denom=max(rms(b), 1e-3))
 
 
-def test_mlp_tensorcore_is_deterministic(ttt):
+@pytest.mark.parametrize("impl", TC_MLP)
+def test_mlp_tensorcore_is_deterministic(ttt, impl):
     w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=256)
     inp = make_inputs(w, 6)
-    a = gpu_mlp(ttt, w, inp, impl="tensorcore")
-    b = gpu_mlp(ttt, w, inp, impl="tensorcore")
+    a = gpu_mlp(ttt, w, inp, impl=impl)
+    b = gpu_mlp(ttt, w, inp, impl=impl)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
 
@@ -380,7 +405,7 @@ def test_mlp_host_buffers_end_to_end(ttt):
         np.testing.assert_array_equal(a.numpy(), b)
 
 
-@pytest.mark.parametrize("impl", ["tensorcore", "generic"])
+@pytest.mark.parametrize("impl", TC_MLP + ["generic"])
 def test_mlp_in_place_state(ttt, impl):
     """Final-state buffers that are the initial-state buffers (in-place update)."""
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=64)
@@ -394,9 +419,10 @@ def test_mlp_in_place_state(ttt, impl):
         np.testing.assert_array_equal(g[name].cpu().numpy(), r)
 
 
+@pytest.mark.parametrize("impl", TC_MLP)
 @pytest.mark.parametrize("kw", [dict(T=40), dict(dtype="f32", T=64)])
-def test_mlp_tensorcore_unsupported_shapes(ttt, kw):
+def test_mlp_tensorcore_unsupported_shapes(ttt, kw, impl):
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=1, **kw)
     with pytest.raises(ttt.TTTError) as ei:
-        gpu_mlp(ttt, w, make_inputs(w, 0), impl="tensorcore")
+        gpu_mlp(ttt, w, make_inputs(w, 0), impl=impl)
     assert ei.value.status == 6
