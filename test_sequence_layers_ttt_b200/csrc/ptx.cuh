@@ -115,6 +115,22 @@ __device__ __forceinline__ void cluster_arrive() {
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
+// wait with cluster-scope acquire, for a barrier completed by another CTA's st.async
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// store into another CTA's shared memory that counts its bytes on that CTA's mbarrier
+// (both addresses from mapa_shared)
+__device__ __forceinline__ void st_async_f32x2(uint32_t addr, float x, float y, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 ::"r"(addr), "f"(x), "f"(y), "r"(remote_bar) : "memory");
+}
 // plain stores into another CTA's shared memory (address from mapa_shared)
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float x, float y) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");

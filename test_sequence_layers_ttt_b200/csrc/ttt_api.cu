@@ -51,9 +51,10 @@ ttt_status finish(cudaError_t launch, cudaStream_t stream) {
     if (launch != cudaSuccess) return TTT_ERR_CUDA;
     if (!check_env()) return TTT_OK;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
-    unsigned int flag = 0;
+    unsigned int flag = 0, mlp_flag = 0;
     if (ttt::read_and_clear_device_error(&flag) != cudaSuccess) return TTT_ERR_CUDA;
-    return flag ? TTT_ERR_TIMEOUT : TTT_OK;
+    if (ttt::read_and_clear_mlp_error(&mlp_flag) != cudaSuccess) return TTT_ERR_CUDA;
+    return (flag | mlp_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
 }
 
 ttt_status validate_linear(const LinearArgs& a) {

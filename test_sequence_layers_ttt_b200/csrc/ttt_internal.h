@@ -44,6 +44,8 @@ cudaError_t launch_mlp_tc(const MlpArgs& a, cudaStream_t stream);
 constexpr int kMlpSplitMaxScans = 74;
 bool mlp_split_supports(const MlpArgs& a);
 cudaError_t launch_mlp_split(const MlpArgs& a, cudaStream_t stream);
+// Error word of the split kernel (a bounded wait on the other CTA gave up).
+cudaError_t read_and_clear_mlp_error(unsigned int* out);
 
 // Device-side error word set by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_device_error(unsigned int* out);

@@ -558,20 +558,45 @@ ttt_mlp_tc_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ Qg,
 //   Hq H^T and Hq W2                                partial sums swapped
 // Both CTAs add the partials in rank order, so their copies of Y, G2, b2 and
 // Z2q agree exactly.  CTA r writes the outputs of tokens [8r, 8r + 8) of each
-// chunk.  Two hardware cluster barriers per chunk order the swaps; the W1 and
-// W2 updates run between the arrive and the wait of the second one.
+// chunk.
+//
+// The fp32 state of the slice stays in registers, one 16 x 64 tile per warp in
+// the mma accumulator layout, so an update is a register add; after each
+// update the warp writes the tile's bf16 hi / lo split to shared memory, where
+// the products read it with ldmatrix.  The Y partials travel by st.async,
+// counted in bytes on the receiver's mbarrier (bounded wait, no fence on the
+// sender); the Hq partials by plain remote stores ordered by a hardware cluster
+// barrier, with the W1 and W2 updates between its arrive and its wait.
 namespace split {
 
 constexpr int kSplit = 2;
 constexpr int HL = HID / kSplit;  // hidden units per CTA
 constexpr int NPL = HL / 64;      // 64-column panels of a [16][HL] activation
 
-// W2^T slice [out][HL], rows XOR-swizzled in 8-float groups
-__device__ __forceinline__ int w2i(int out, int hid) { return out * HL + ((((hid >> 3) ^ (out & 7))) << 3) + (hid & 7); }
+// byte offset in a bf16 W2^T slice tile [out][HL] (256-byte rows, 16-byte groups XOR-swizzled)
+__device__ __forceinline__ uint32_t w2b(int out, int hid) {
+    return out * (HL * 2) + ((((hid >> 3) ^ (out & 7))) << 4) + (hid & 7) * 2;
+}
+// W1 as the B operand of [16 x in] x W1 (k = inputs 16ks.., n = hidden 8hb..), from the
+// bf16 W1^T slice tiles [hid][in] (128-byte rows, swizzled like the activation tiles)
+__device__ __forceinline__ void ld_w1(uint32_t wh, uint32_t wl, int ks, int hb, int lane, uint32_t (&b)[4]) {
+    const int mi = lane >> 3, r = lane & 7;
+    ptx::ldsm_x4((mi >> 1 ? wl : wh) + swz(8 * hb + r, 16 * ks + 8 * (mi & 1)), b[0], b[1], b[2], b[3]);
+}
+// W2 as the B operand of [16 x hid] x W2 (k = hidden 16ks.., n = outputs 8ot..): hi k-halves, lo k-halves
+__device__ __forceinline__ void ld_w2_kh(uint32_t wh, uint32_t wl, int ks, int ot, int lane, uint32_t (&b)[4]) {
+    const int mi = lane >> 3, r = lane & 7;
+    ptx::ldsm_x4((mi >> 1 ? wl : wh) + w2b(8 * ot + r, 16 * ks + 8 * (mi & 1)), b[0], b[1], b[2], b[3]);
+}
+// W2^T as the B operand of [16 x out] x W2^T (k = outputs 16ks.., n = hidden 8hb..)
+__device__ __forceinline__ void ld_w2_ko(uint32_t wh, uint32_t wl, int ks, int hb, int lane, uint32_t (&b)[4]) {
+    const int mi = lane >> 3, r = lane & 7;
+    ptx::ldsm_x4_t((mi >> 1 ? wl : wh) + w2b(16 * ks + 8 * (mi & 1) + r, 8 * hb), b[0], b[1], b[2], b[3]);
+}
 
 struct Smem {
-    float w1t[HL * D];  // W1^T slice [hid][in], swizzled with w1i
-    float w2t[D * HL];  // W2^T slice [out][hid], swizzled with w2i
+    unsigned char w1h[HL * D * 2], w1l[HL * D * 2];  // W1^T slice [hid][in] as bf16 hi / lo, swizzled with swz
+    unsigned char w2h[D * HL * 2], w2l[D * HL * 2];  // W2^T slice [out][hid] as bf16 hi / lo, swizzled with w2b
     float b1[HL], b2[D];
     float gam[D], bet[D];
     unsigned char K[PANEL], V[PANEL], Q[PANEL];
@@ -587,7 +612,31 @@ struct Smem {
     uint4 afrag[2][32];
     float4 a2p[kSplit * NPL][2][32];  // Hq H^T partial of CTA r, panel p at [NPL r + p]
     alignas(16) float eta[kChunk];
+    uint64_t ybar;   // completes when the other CTA's Y partial of the chunk has landed in yp
+    int abort_flag;  // set after a wait gave up (in both CTAs)
 };
+
+constexpr uint32_t kYBytes = kChunk * D * 4;   // one CTA's Y partial
+constexpr long long kTimeoutCycles = 2000000000LL;
+__device__ unsigned int g_mlp_error_word = 0;
+
+// bounded wait on a barrier completed by the other CTA's stores; false once the
+// wait has given up here or in the other CTA (then both run on without waiting)
+__device__ __forceinline__ bool wait_peer(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t peer_abort_flag) {
+    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (int spins = 1;; spins++) {
+        if (*abort_flag) return false;
+        if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+        if ((spins & 63) == 0 && clock64() - t0 > kTimeoutCycles) {
+            *abort_flag = 1;
+            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort_flag), "r"(1u) : "memory");
+            atomicOr(&g_mlp_error_word, 1u);
+            return false;
+        }
+    }
+}
 
 // d_h += ah bh, d_l += ah bl + al bh: the split product in two accumulators
 __device__ __forceinline__ void mma3s(float (&dh)[4], float (&dl)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
@@ -618,20 +667,54 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
     const int hid0 = HL * (int)rank;  // first hidden unit of this CTA's slice
     auto remote = [&](const void* p) { return ptx::mapa_shared(ptx::smem_addr(p), peer); };
 
-    // ---- initial state: this CTA's slice of W1, b1, W2; all of b2
-    for (int i = tid; i < D * HL; i += kThreads) {
-        const int in = i / HL, hl = i % HL;  // W1_0 [in][hid]
-        s.w1t[w1i(hl, in)] = W1_0[bh * D * HID + (long)in * HID + hid0 + hl];
-    }
-    for (int i = tid; i < HL * D; i += kThreads) {
-        const int hl = i / D, out = i % D;  // W2_0 [hid][out]
-        s.w2t[split::w2i(out, hl)] = W2_0[bh * HID * D + (long)(hid0 + hl) * D + out];
-    }
+    // ---- initial state.  The fp32 state lives in registers, one 16 x 64 tile per warp in
+    // the mma accumulator layout: warp w < 8 holds W1^T rows (hidden) [16w, 16w + 16),
+    // warp 8 + v holds W2^T rows (outputs) [16 (v & 3), +16) x hidden [64 (v >> 2), +64).
+    // Element sr[jp][nt][2 rh + e] sits at row 16 m + g + 8 rh, column 16 jp + 8 nt + 2 t + e.
+    // Shared memory holds the bf16 hi / lo copies the products read.
+    float sr[4][2][4];
+    const bool w1_warp = warp < 8;
+    const int vw = warp & 7, mo = vw & 3, pp = vw >> 2;
+    auto state_index = [&](int jp, int nt, int rh, int e) -> long {
+        if (w1_warp) {  // W1_0 [in][hid]
+            const int hid = 16 * vw + g + 8 * rh, in = 16 * jp + 8 * nt + 2 * t + e;
+            return bh * D * HID + (long)in * HID + hid0 + hid;
+        }
+        const int out = 16 * mo + g + 8 * rh, hid = 64 * pp + 16 * jp + 8 * nt + 2 * t + e;  // W2_0 [hid][out]
+        return bh * HID * D + (long)(hid0 + hid) * D + out;
+    };
+    // bf16 hi / lo copy of the pair sr[jp][nt][2 rh], sr[jp][nt][2 rh + 1]
+    auto store_split = [&](int jp, int nt, int rh, float x0, float x1) {
+        uint32_t hi, lo;
+        ptx::split_pair(x0, x1, hi, lo);
+        const uint32_t off = w1_warp ? swz(16 * vw + g + 8 * rh, 16 * jp + 8 * nt + 2 * t)
+                                     : split::w2b(16 * mo + g + 8 * rh, 64 * pp + 16 * jp + 8 * nt + 2 * t);
+        unsigned char* th = w1_warp ? s.w1h : s.w2h;
+        unsigned char* tl = w1_warp ? s.w1l : s.w2l;
+        *reinterpret_cast<uint32_t*>(th + off) = hi;
+        *reinterpret_cast<uint32_t*>(tl + off) = lo;
+    };
+#pragma unroll
+    for (int jp = 0; jp < 4; jp++)
+#pragma unroll
+        for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+            for (int rh = 0; rh < 2; rh++) {
+                const float* W0 = w1_warp ? W1_0 : W2_0;
+                sr[jp][nt][2 * rh] = W0[state_index(jp, nt, rh, 0)];
+                sr[jp][nt][2 * rh + 1] = W0[state_index(jp, nt, rh, 1)];
+                store_split(jp, nt, rh, sr[jp][nt][2 * rh], sr[jp][nt][2 * rh + 1]);
+            }
     for (int i = tid; i < HL; i += kThreads) s.b1[i] = b1_0[bh * HID + hid0 + i];
     if (tid < D) {
         s.b2[tid] = b2_0[bh * D + tid];
         s.gam[tid] = gamma[(long)h * D + tid];
         s.bet[tid] = beta[(long)h * D + tid];
+    }
+    if (tid == 0) {
+        ptx::mbar_init(&s.ybar, 1);
+        s.abort_flag = 0;
+        ptx::fence_mbar_init();
     }
 
     // ---- token loads (both CTAs read the whole chunk): as in the one-CTA kernel
@@ -647,17 +730,23 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
     if (n > 0) fetch(0);
 
     const uint32_t sK = ptx::smem_addr(s.K), sQ = ptx::smem_addr(s.Q);
+    const uint32_t sW2h = ptx::smem_addr(s.w2h), sW2l = ptx::smem_addr(s.w2l);
+    const uint32_t sW1h = ptx::smem_addr(s.w1h), sW1l = ptx::smem_addr(s.w1l);
     float* Zbh = Z + tok0 * D;
     // this warp's hidden units [8 warp, 8 warp + 8): panel and column inside it
     const int p = warp >> 3, pc = 8 * (warp & 7) + 2 * t;
 
-    // the peer CTA is running before any store reaches its shared memory
+    // the peer CTA is running, its barrier initialised, before any store reaches its shared memory
     ptx::cluster_arrive();
     ptx::cluster_wait();
+    const uint32_t ybar_peer = remote(&s.ybar), abort_peer = remote(&s.abort_flag);
 
     for (int c = 0; c < n; c++) {
         // ================================================= phase 0: this chunk's tokens in, next chunk's requested
         __syncthreads();
+        // after an abort neither CTA arms its barrier or sends, so no byte count runs away
+        const bool live = !*reinterpret_cast<volatile int*>(&s.abort_flag);
+        if (tid == 0 && live) ptx::mbar_arrive_expect_tx(&s.ybar, split::kYBytes);
         if (tid < 384) {
             unsigned char* dst = lt == 0 ? s.K : (lt == 1 ? s.V : s.Q);
             *reinterpret_cast<uint4*>(dst + swz_chunk(lrow, lchunk)) = pf;
@@ -681,16 +770,12 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 uint32_t ax[4], aq[4];
                 ld_a(sK, ks, lane, ax);
                 ld_a(sQ, ks, lane, aq);
-                const int hid = 8 * warp + g, in = 16 * ks + 2 * t;
-                const float2 w0 = *reinterpret_cast<const float2*>(&s.w1t[w1i(hid, in)]);
-                const float2 w1 = *reinterpret_cast<const float2*>(&s.w1t[w1i(hid, in + 8)]);
-                uint32_t bh0, bl0, bh1, bl1;
-                ptx::split_pair(w0.x, w0.y, bh0, bl0);
-                ptx::split_pair(w1.x, w1.y, bh1, bl1);
-                mma(z1, ax, bh0, bh1);
-                mma(z1l, ax, bl0, bl1);
-                mma(zq, aq, bh0, bh1);
-                mma(zql, aq, bl0, bl1);
+                uint32_t b[4];
+                split::ld_w1(sW1h, sW1l, ks, warp, lane, b);
+                mma(z1, ax, b[0], b[1]);
+                mma(z1l, ax, b[2], b[3]);
+                mma(zq, aq, b[0], b[1]);
+                mma(zql, aq, b[2], b[3]);
             }
             float hv[4];
 #pragma unroll
@@ -715,14 +800,10 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 uint32_t ah[4], al[4];
                 ld_a(ptx::smem_addr(s.Hh[ks >> 2]), ks & 3, lane, ah);
                 ld_a(ptx::smem_addr(s.Hl[ks >> 2]), ks & 3, lane, al);
-                const int out = 8 * warp + g, hid = 16 * ks + 2 * t;
-                const float2 w0 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid)]);
-                const float2 w1 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid + 8)]);
-                uint32_t bh0, bl0, bh1, bl1;
-                ptx::split_pair(w0.x, w0.y, bh0, bl0);
-                ptx::split_pair(w1.x, w1.y, bh1, bl1);
-                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, bh0, bh1, bl0, bl1);
-                else split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+                uint32_t b[4];
+                split::ld_w2_kh(sW2h, sW2l, ks, warp, lane, b);
+                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, b[0], b[1], b[2], b[3]);
+                else split::mma3s(acc, accl, ah, al, b[0], b[1], b[2], b[3]);
             }
 #pragma unroll
             for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) + (acc2[r] + acc2l[r]);
@@ -731,8 +812,10 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
             float* y1 = &s.yp[rank][(g + 8) * YLD + col];
             *reinterpret_cast<float2*>(y0) = make_float2(acc[0], acc[1]);
             *reinterpret_cast<float2*>(y1) = make_float2(acc[2], acc[3]);
-            ptx::st_cluster_f32x2(remote(y0), acc[0], acc[1]);
-            ptx::st_cluster_f32x2(remote(y1), acc[2], acc[3]);
+            if (live) {
+                ptx::st_async_f32x2(remote(y0), acc[0], acc[1], ybar_peer);
+                ptx::st_async_f32x2(remote(y1), acc[2], acc[3], ybar_peer);
+            }
         } else {
             if (warp == 8) {
                 // A = tril(eta_s (q_t . x_s + 1)) as -A hi/lo A fragments
@@ -764,8 +847,8 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 *reinterpret_cast<uint32_t*>(s.EXl + swz(row, col)) = lo;
             }
         }
-        ptx::cluster_arrive();
-        ptx::cluster_wait();
+        __syncthreads();
+        split::wait_peer(&s.ybar, (uint32_t)(c & 1), &s.abort_flag, abort_peer);
 
         // ================================================= phase 3: Y = b2 + partials, G2 = dl/dY, E2 = -eta G2 (warp w: token w)
         {
@@ -807,11 +890,9 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 uint32_t ah[4], al[4];
                 ld_a(g2h, ks, lane, ah);
                 ld_a(g2l, ks, lane, al);
-                const int hid = 8 * warp + g, out = 16 * ks + 2 * t;
-                uint32_t bh0, bl0, bh1, bl1;
-                ptx::split_pair(s.w2t[split::w2i(out, hid)], s.w2t[split::w2i(out + 1, hid)], bh0, bl0);
-                ptx::split_pair(s.w2t[split::w2i(out + 8, hid)], s.w2t[split::w2i(out + 9, hid)], bh1, bl1);
-                split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+                uint32_t b[4];
+                split::ld_w2_ko(sW2h, sW2l, ks, warp, lane, b);
+                split::mma3s(acc, accl, ah, al, b[0], b[1], b[2], b[3]);
             }
 #pragma unroll
             for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) * gelu_prime_sig(z1[r], sg1[r]);
@@ -871,14 +952,10 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 uint32_t ah[4], al[4];
                 ld_a(ptx::smem_addr(s.Hqh[ks >> 2]), ks & 3, lane, ah);
                 ld_a(ptx::smem_addr(s.Hql[ks >> 2]), ks & 3, lane, al);
-                const int out = 8 * ot + g, hid = 16 * ks + 2 * t;
-                const float2 w0 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid)]);
-                const float2 w1 = *reinterpret_cast<const float2*>(&s.w2t[split::w2i(out, hid + 8)]);
-                uint32_t bh0, bl0, bh1, bl1;
-                ptx::split_pair(w0.x, w0.y, bh0, bl0);
-                ptx::split_pair(w1.x, w1.y, bh1, bl1);
-                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, bh0, bh1, bl0, bl1);
-                else split::mma3s(acc, accl, ah, al, bh0, bh1, bl0, bl1);
+                uint32_t b[4];
+                split::ld_w2_kh(sW2h, sW2l, ks, ot, lane, b);
+                if (ks & 1) split::mma3s(acc2, acc2l, ah, al, b[0], b[1], b[2], b[3]);
+                else split::mma3s(acc, accl, ah, al, b[0], b[1], b[2], b[3]);
             }
 #pragma unroll
             for (int r = 0; r < 4; r++) acc[r] = (acc[r] + accl[r]) + (acc2[r] + acc2l[r]);
@@ -916,11 +993,9 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                     for (int rh = 0; rh < 2; rh++) {
-                        float2* wp = reinterpret_cast<float2*>(&s.w1t[w1i(16 * mt + g + 8 * rh, 16 * jp + 8 * nt + 2 * t)]);
-                        float2 wv = *wp;
-                        wv.x += d[nt][2 * rh];
-                        wv.y += d[nt][2 * rh + 1];
-                        *wp = wv;
+                        sr[jp][nt][2 * rh] += d[nt][2 * rh];
+                        sr[jp][nt][2 * rh + 1] += d[nt][2 * rh + 1];
+                        store_split(jp, nt, rh, sr[jp][nt][2 * rh], sr[jp][nt][2 * rh + 1]);
                     }
             }
             float db[4];
@@ -932,7 +1007,6 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
             }
         } else {
             // W2^T[out][hid] += E2^T H; output rows [16 mo, 16 mo + 16), hidden panel pp
-            const int v = warp - 8, mo = v & 3, pp = v >> 2;
             uint32_t ah[4], al[4];
             ld_a_t(ptx::smem_addr(s.E2h), mo, lane, ah);
             ld_a_t(ptx::smem_addr(s.E2l), mo, lane, al);
@@ -950,12 +1024,9 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
                 for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                     for (int rh = 0; rh < 2; rh++) {
-                        float2* wp = reinterpret_cast<float2*>(
-                            &s.w2t[split::w2i(16 * mo + g + 8 * rh, 64 * pp + 16 * jp + 8 * nt + 2 * t)]);
-                        float2 wv = *wp;
-                        wv.x += d[nt][2 * rh];
-                        wv.y += d[nt][2 * rh + 1];
-                        *wp = wv;
+                        sr[jp][nt][2 * rh] += d[nt][2 * rh];
+                        sr[jp][nt][2 * rh + 1] += d[nt][2 * rh + 1];
+                        store_split(jp, nt, rh, sr[jp][nt][2 * rh], sr[jp][nt][2 * rh + 1]);
                     }
             }
         }
@@ -1024,16 +1095,26 @@ ttt_mlp_split_kernel(int T, int H, float eps, const __nv_bfloat16* __restrict__ 
             }
         }
     }
-    __syncthreads();
-    // ---- final state: this CTA's slice; CTA 0 writes b2
-    for (int i = tid; i < D * HL; i += kThreads) {
-        const int in = i / HL, hl = i % HL;
-        W1_T[bh * D * HID + (long)in * HID + hid0 + hl] = s.w1t[w1i(hl, in)];
+    // no CTA leaves while the other may still store into its shared memory; after an
+    // abort, stores already sent get time to land first
+    if (*reinterpret_cast<volatile int*>(&s.abort_flag)) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 200000) {
+        }
     }
-    for (int i = tid; i < HL * D; i += kThreads) {
-        const int hl = i / D, out = i % D;
-        W2_T[bh * HID * D + (long)(hid0 + hl) * D + out] = s.w2t[split::w2i(out, hl)];
-    }
+    ptx::cluster_arrive();
+    ptx::cluster_wait();
+    // ---- final state: this CTA's slice from the registers; CTA 0 writes b2
+#pragma unroll
+    for (int jp = 0; jp < 4; jp++)
+#pragma unroll
+        for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+            for (int rh = 0; rh < 2; rh++) {
+                float* WT = w1_warp ? W1_T : W2_T;
+                WT[state_index(jp, nt, rh, 0)] = sr[jp][nt][2 * rh];
+                WT[state_index(jp, nt, rh, 1)] = sr[jp][nt][2 * rh + 1];
+            }
     for (int i = tid; i < HL; i += kThreads) b1_T[bh * HID + hid0 + i] = s.b1[i];
     if (rank == 0 && tid < D) b2_T[bh * D + tid] = s.b2[tid];
 }
@@ -1058,6 +1139,13 @@ cudaError_t launch_mlp_tc(const MlpArgs& a, cudaStream_t stream) {
 }
 
 bool mlp_split_supports(const MlpArgs& a) { return mlp_tc_supports(a); }
+
+cudaError_t read_and_clear_mlp_error(unsigned int* out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, split::g_mlp_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(split::g_mlp_error_word, &zero, sizeof(unsigned int));
+}
 
 cudaError_t launch_mlp_split(const MlpArgs& a, cudaStream_t stream) {
     if (!mlp_split_supports(a)) return cudaErrorInvalidValue;
