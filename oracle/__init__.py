@@ -42,6 +42,9 @@ def _load():
             f = getattr(lib, "oracle_ttt_linear" + sfx)
             f.restype = I
             f.argtypes = [I, I, I, I, I, I, real] + [P] * 11 + [I]
+            f = getattr(lib, "oracle_ttt_linear_decode" + sfx)
+            f.restype = I
+            f.argtypes = [I, I, I, I, I, I, I, real] + [P] * 11 + [I]
             f = getattr(lib, "oracle_ttt_mlp" + sfx)
             f.restype = I
             f.argtypes = [I, I, I, I, I, I, real] + [P] * 15 + [I]
@@ -92,6 +95,34 @@ def ttt_linear(Q, K, V, eta, W0, b0, gamma, beta, mini_batch: int,
     if rc != 0:
         raise ValueError("oracle_ttt_linear: bad arguments")
     return Z, W_T, b_T
+
+
+def ttt_linear_decode(Q, K, V, eta, W, b, W_mb, b_mb, gamma, beta, mini_batch: int, pos0: int,
+                      mode: int = MODE_LN_RESIDUAL, ln_eps: float = 1e-6,
+                      precision: str = "f64", threads: Optional[int] = None):
+    """TTT-Linear scan continued by T tokens from position pos0 of a mini-batch.
+
+    W, b: running state [B,H,d,d], [B,H,d]; W_mb, b_mb: state the current
+    mini-batch started from (read when pos0 > 0).  Returns (Z, W, b, W_mb,
+    b_mb) after the T tokens; W_mb, b_mb are then the start state of the
+    mini-batch the next token falls in.  The inputs are not modified."""
+    dt = np.float64 if precision == "f64" else np.float32
+    Q, K, V, eta = (_arr(x, dt) for x in (Q, K, V, eta))
+    B, H, T, d = Q.shape
+    W = _arr(W, dt).copy()
+    W_mb = _arr(W_mb, dt).copy() if W_mb is not None else W.copy()
+    b = _arr(b, dt).copy() if b is not None else np.zeros((B, H, d), dt)
+    b_mb = _arr(b_mb, dt).copy() if b_mb is not None else b.copy()
+    gamma = _arr(gamma, dt) if gamma is not None else np.ones((H, d), dt)
+    beta = _arr(beta, dt) if beta is not None else np.zeros((H, d), dt)
+    Z = np.zeros((B, H, T, d), dt)
+    fn = getattr(_load(), "oracle_ttt_linear_decode_" + precision)
+    rc = fn(B, H, T, d, int(mini_batch), int(pos0), int(mode), ln_eps, _ptr(Q), _ptr(K), _ptr(V),
+            _ptr(eta), _ptr(W), _ptr(b), _ptr(W_mb), _ptr(b_mb), _ptr(gamma), _ptr(beta), _ptr(Z),
+            _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_ttt_linear_decode: bad arguments")
+    return Z, W, b, W_mb, b_mb
 
 
 def ttt_mlp(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, gamma, beta, mini_batch: int,

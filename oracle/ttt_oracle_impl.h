@@ -201,6 +201,63 @@ int FN(oracle_ttt_linear)(int B, int H, int T, int d, int mb, int mode, REAL eps
     return 0;
 }
 
+/*
+ * TTT-Linear decode: the same scan continued by T more tokens from position
+ * pos0 of a mini-batch [LR1], [LR5].  The state carried between calls is the
+ * running state (Wc, bc) = W_t and the state the current mini-batch started
+ * from (Wm, bm), at which that mini-batch's gradients are taken.  All four are
+ * read and overwritten in place; on return (Wm, bm) is the start state of the
+ * mini-batch the next token falls in.  bc / bm may be NULL in plain mode.
+ * Returns 0, or -1 on bad arguments.
+ */
+int FN(oracle_ttt_linear_decode)(int B, int H, int T, int d, int mb, int pos0, int mode, REAL eps,
+                                 const REAL* Q, const REAL* K, const REAL* V, const REAL* eta,
+                                 REAL* Wc_all, REAL* bc_all, REAL* Wm_all, REAL* bm_all,
+                                 const REAL* gamma, const REAL* beta, REAL* Z, int nthreads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || mb <= 0 || pos0 < 0 || pos0 >= mb) return -1;
+    if (mode != ORACLE_MODE_PLAIN && mode != ORACLE_MODE_LN_RESIDUAL) return -1;
+    if (nthreads <= 0) nthreads = 1;
+    const int ln = mode != ORACLE_MODE_PLAIN;
+    long nbh = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < nbh; bh++) {
+        int h = (int)(bh % H);
+        const REAL* gam = gamma ? gamma + (long)h * d : NULL;
+        const REAL* bet = beta ? beta + (long)h * d : NULL;
+        REAL* Wc = Wc_all + bh * d * d;
+        REAL* Wm = Wm_all + bh * d * d;
+        REAL* buf = (REAL*)calloc((size_t)6 * d, sizeof(REAL));
+        REAL *bc = buf, *bm = buf + d, *g = buf + 2 * d, *scratch = buf + 3 * d;
+        if (ln && bc_all) memcpy(bc, bc_all + bh * d, sizeof(REAL) * d);
+        if (ln && bm_all) memcpy(bm, bm_all + bh * d, sizeof(REAL) * d);
+        for (int t = 0; t < T; t++) {
+            if ((pos0 + t) % mb == 0) { /* a mini-batch starts at this token */
+                memcpy(Wm, Wc, sizeof(REAL) * (size_t)d * d);
+                memcpy(bm, bc, sizeof(REAL) * d);
+            }
+            long row = (bh * T + t) * d;
+            REAL e = eta[bh * T + t];
+            FN(linear_token_dy)(d, mode, eps, K + row, V + row, Wm, bm, gam, bet, g, scratch);
+            for (int i = 0; i < d; i++) {
+                REAL ek = e * K[row + i];
+                REAL* Wi = Wc + (long)i * d;
+                for (int j = 0; j < d; j++) Wi[j] -= ek * g[j];
+            }
+            if (ln)
+                for (int j = 0; j < d; j++) bc[j] -= e * g[j];
+            FN(linear_apply)(d, mode, eps, Q + row, Wc, bc, gam, bet, Z + row, scratch);
+        }
+        if ((pos0 + T) % mb == 0) { /* the next token starts a mini-batch */
+            memcpy(Wm, Wc, sizeof(REAL) * (size_t)d * d);
+            memcpy(bm, bc, sizeof(REAL) * d);
+        }
+        if (ln && bc_all) memcpy(bc_all + bh * d, bc, sizeof(REAL) * d);
+        if (ln && bm_all) memcpy(bm_all + bh * d, bm, sizeof(REAL) * d);
+        free(buf);
+    }
+    return 0;
+}
+
 /* ----------------------------- TTT-MLP ------------------------------------ */
 
 static REAL FN(gelu)(REAL x) {

@@ -457,6 +457,89 @@ def test_golden_regression_linear_tiny():
 # The pins catch plausible mistakes (mutations planted in a copy of the oracle)
 # ----------------------------------------------------------------------------
 
+# ----------------------------------------------------------------------------
+# Decode: the scan continued from the middle of a mini-batch (Key takeaways,
+# bullets 1 and 5), state carried between calls
+# ----------------------------------------------------------------------------
+
+def decode_in_pieces(Q, K, V, eta, W0, b0, gamma, beta, mb, cuts, mode=LN):
+    """Run the oracle's decode over [0, T) in the pieces given by `cuts`,
+    carrying (W, b, W_mb, b_mb) from call to call."""
+    T = Q.shape[2]
+    W, b, W_mb, b_mb = W0, b0, None, None
+    Zs = []
+    bounds = [0, *cuts, T]
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = (slice(None), slice(None), slice(a, c))
+        Z, W, b, W_mb, b_mb = oracle.ttt_linear_decode(Q[sl], K[sl], V[sl], eta[sl], W, b, W_mb, b_mb,
+                                                       gamma, beta, mb, a % mb, mode)
+        Zs.append(Z)
+    return np.concatenate(Zs, axis=2), W, b, W_mb, b_mb
+
+
+@pytest.mark.parametrize("mode,mb,cuts", [
+    (LN, 16, [5, 6, 21, 40]),   # ragged pieces, several inside one mini-batch
+    (LN, 8, [1, 2, 3, 19, 33]),
+    (LN, 48, [7, 30]),          # one mini-batch for the whole stream
+    (PLAIN, 16, [3, 17, 18]),
+    (LN, 1, [4, 9]),            # b = 1: online GD
+])
+def test_decode_pieces_equal_minibatch_rule(mode, mb, cuts):
+    """Decode calls split anywhere reproduce the mini-batch rule written out with
+    torch autograd over the whole stream."""
+    Q, K, V, eta, W0, b0, gamma, beta = small_linear_case(3, T=48, mode=mode)
+    Z, W, b, _, _ = decode_in_pieces(Q, K, V, eta, W0, b0, gamma, beta, mb, cuts, mode)
+    fn = (lambda x, W_, b_: f_linear(x, W_, b_, t64(gamma[0]), t64(beta[0]), mode))
+    Zr, (Wr, br) = minibatch_restatement(fn, [t64(W0[0, 0]), t64(b0[0, 0])], t64(Q[0, 0]),
+                                         t64(K[0, 0]), t64(V[0, 0]), t64(eta[0, 0]), mb)
+    assert rel(Z[0, 0], Zr.numpy()) < 1e-11
+    assert rel(W[0, 0], Wr.numpy()) < 1e-11
+    if mode == LN:
+        assert rel(b[0, 0], br.numpy()) < 1e-11
+
+
+def test_decode_single_tokens_theorem1():
+    """Token-by-token decode in plain mode, one mini-batch over the whole stream,
+    eta = 1/2, W0 = 0: z_t = sum_{s<=t} (q_t . k_s) v_s (Theorem 1), and the
+    mini-batch start state stays at W0 until the stream's mini-batch ends."""
+    r = rng(11)
+    T, d = 24, 8
+    Q, K, V = (r.normal(0, 1, (1, 1, T, d)) for _ in range(3))
+    eta = np.full((1, 1, T), 0.5)
+    W, W_mb = np.zeros((1, 1, d, d)), None
+    Z = np.zeros((1, 1, T, d))
+    for t in range(T):
+        sl = (slice(None), slice(None), slice(t, t + 1))
+        Z[sl], W, _, W_mb, _ = oracle.ttt_linear_decode(Q[sl], K[sl], V[sl], eta[sl], W, None, W_mb, None,
+                                                        None, None, T, t, PLAIN)
+        if t < T - 1:
+            assert not np.any(W_mb)
+    S = np.tril(Q[0, 0] @ K[0, 0].T)
+    assert rel(Z[0, 0], S @ V[0, 0]) < 1e-12
+    assert rel(W_mb[0, 0], K[0, 0].T @ V[0, 0]) < 1e-12  # the next mini-batch starts from W_T
+
+
+def test_decode_empty_call_keeps_state():
+    Q, K, V, eta, W0, b0, gamma, beta = small_linear_case(4, T=8)
+    Wm = W0 + 0.25
+    e = (slice(None), slice(None), slice(0, 0))
+    Z, W, b, W_mb, b_mb = oracle.ttt_linear_decode(Q[e], K[e], V[e], eta[e], W0, b0, Wm, b0 * 2,
+                                                   gamma, beta, 16, 5)
+    assert Z.shape == (1, 1, 0, 8)
+    np.testing.assert_array_equal(W, W0)
+    np.testing.assert_array_equal(W_mb, Wm)  # mid-mini-batch: its start state is kept
+    np.testing.assert_array_equal(b_mb, b0 * 2)
+    _, W, _, W_mb, _ = oracle.ttt_linear_decode(Q[e], K[e], V[e], eta[e], W0, b0, Wm, b0, gamma, beta, 16, 0)
+    np.testing.assert_array_equal(W_mb, W0)  # at a boundary the next mini-batch starts from W
+
+
+@pytest.mark.parametrize("pos0", [-1, 16])
+def test_decode_rejects_bad_position(pos0):
+    Q, K, V, eta, W0, b0, gamma, beta = small_linear_case(4, T=8)
+    with pytest.raises(ValueError):
+        oracle.ttt_linear_decode(Q, K, V, eta, W0, b0, W0, b0, gamma, beta, 16, pos0)
+
+
 MUTATIONS = {
     "drop_mean_term": ("g[j] = s * (g[j] - mean_gx - xhat[j] * mean_gxx);",
                        "g[j] = s * (g[j] - xhat[j] * mean_gxx);"),
@@ -477,6 +560,12 @@ MUTATIONS = {
         "(REAL)0.5 * x * ((REAL)1 - th * th) * c * ((REAL)1 + (REAL)3 * (REAL)0.044715 * x * x);",
         "(REAL)0.5 * x * ((REAL)1 - th * th) * c;"),
     "mlp_bias_not_updated": ("for (int j = 0; j < hid; j++) b1c[j] -= e * g1[j];", ""),
+    "decode_gradient_at_running_state": (
+        "FN(linear_token_dy)(d, mode, eps, K + row, V + row, Wm, bm, gam, bet, g, scratch);",
+        "FN(linear_token_dy)(d, mode, eps, K + row, V + row, Wc, bc, gam, bet, g, scratch);"),
+    "decode_no_minibatch_restart": (
+        "if ((pos0 + t) % mb == 0) { /* a mini-batch starts at this token */",
+        "if (0) {"),
 }
 
 
@@ -525,6 +614,8 @@ def _run_pins_with(lib_path):
         lambda: test_b1_equals_online_gd(LN),
         lambda: test_minibatch_rule_linear(LN, 8, 48),
         lambda: test_minibatch_rule_mlp(8, 24),
+        lambda: test_decode_pieces_equal_minibatch_rule(LN, 8, [1, 2, 3, 19, 33]),
+        test_decode_single_tokens_theorem1,
     ]
     try:
         for pin in pins:
