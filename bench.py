@@ -40,6 +40,8 @@ METRIC = "TTT forward tokens/sec on 1 B200 (1.3B-layer shape, 32k ctx); % of roo
 def metric_name(w) -> str:
     if w.name == "linear_1p3b_32k":
         return METRIC
+    if w.name == "decode_1p3b":
+        return "TTT-Linear decode tokens/sec on 1 B200 (1.3B-layer shape, one token per sequence per step)"
     shape = {"linear_125m_2k": "125M-layer shape, 2k ctx", "mlp_8k": "TTT-MLP layer, 8k ctx"}[w.name]
     return f"TTT forward tokens/sec on 1 B200 ({shape}); % of roofline"
 FALLBACK_HBM_GBS = 6650.0
@@ -85,6 +87,7 @@ KERNEL_SOURCES = {
     "ttt_mlp_tc_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_split_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_generic_kernel": ("ttt_mlp_generic.cu", "common.cuh", "ttt_internal.h"),
+    "ttt_linear_decode_kernel": ("ttt_linear_decode.cu", "common.cuh", "ttt_internal.h"),
 }
 
 
@@ -237,18 +240,51 @@ def cpu_oracle_sample(w, inp, target_s: float):
                       f"{dt:.2f} s; tokens counted as scans*T/H"}
 
 
+def decode_state_bytes(w) -> int:
+    """Algorithmic bytes of one decode step (one token for every (batch, head)
+    stream): running state W, b read and written, the mini-batch start state
+    W_mb, b_mb read and written, and the token's q, k, v, eta in and z out."""
+    state = 4 * (w.d * w.d + w.d)
+    es = 2 if w.dtype == "bf16" else 4
+    return w.B * w.H * (4 * state + 3 * w.d * es + 4 + w.d * 4)
+
+
+def cpu_oracle_decode_sample(w, inp, target_s: float):
+    """Time the float64 oracle's decode, one token per (batch, head) stream per
+    step over the whole B x H batch, for about target_s seconds; tokens/s
+    counts one token per sequence per step (B per step)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    W, b, W_mb, b_mb = inp["W0"], inp["b0"], None, None
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        i = steps % w.T
+        sl = {k: inp[k][:, :, i:i + 1] for k in ("Q", "K", "V", "eta")}
+        _, W, b, W_mb, b_mb = oracle.ttt_linear_decode(sl["Q"], sl["K"], sl["V"], sl["eta"], W, b, W_mb, b_mb,
+                                                       inp["gamma"], inp["beta"], w.mini_batch,
+                                                       i % w.mini_batch, w.mode, w.ln_eps, threads=cores)
+        steps += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            break
+    return {"value": steps * w.B / dt, "unit": "tokens/s", "cores": min(cores, w.B * w.H), "kind": "oracle",
+            "sample": f"{steps} single-token decode steps of all {w.B * w.H} (batch, head) streams, "
+                      f"float64 primal oracle, {dt:.2f} s"}
+
+
 def run_reference(args, world, rank):
     w = WORKLOADS[args.workload]
     if rank != 0:
         return
     inp = make_inputs(w, args.seed)
+    sample = cpu_oracle_decode_sample if args.workload == "decode_1p3b" else cpu_oracle_sample
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, inp, 0.5)
+        sample(w, inp, 0.5)
     vals, samples = [], None
     t_start = time.perf_counter()
     per_step = min(args.ref_seconds, 150.0 / max(args.steps, 1))  # whole run within a few minutes
     for _ in range(args.steps):
-        r = cpu_oracle_sample(w, inp, per_step)
+        r = sample(w, inp, per_step)
         vals.append(r["value"])
         samples = r
     elapsed = time.perf_counter() - t_start
@@ -268,6 +304,12 @@ def run_reference(args, world, rank):
 
 
 def workload_config(w):
+    if w.name == "decode_1p3b":
+        return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "mini_batch": w.mini_batch,
+                "qkv_dtype": w.dtype, "state_dtype": "f32", "inner_model": "x + LN(xW + b)",
+                "step": "one token for each of the B x H streams; positions cycle through the mini-batch",
+                "timed": "steps rounded up to whole mini-batch cycles",
+                "l2": "no flush: the 4.3 MB state stays in L2 between steps, as in a decode loop"}
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "mini_batch": w.mini_batch,
             "qkv_dtype": w.dtype, "state_dtype": "f32",
             "inner_model": (f"x + LN(MLP {w.d}->{w.hidden}->{w.d}, GELU)" if w.kind == "mlp"
@@ -275,10 +317,113 @@ def workload_config(w):
             "l2": "inputs (Q/K/V/eta) larger than the 126 MB L2; no flush"}
 
 
+def run_decode(args, world, rank, local):
+    """Single-token decode steps through ttt_linear_decode (d = 64: the decode
+    kernel with the state in registers)."""
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    host = make_inputs(w, args.seed + rank)
+    n_tok = w.T
+    toks = [{k: host[k][:, :, i:i + 1].contiguous().to(dev) for k in ("Q", "K", "V", "eta")}
+            for i in range(n_tok)]
+    gam, bet = host["gamma"].to(dev), host["beta"].to(dev)
+    W, b = host["W0"].to(dev), host["b0"].to(dev)
+    W_mb, b_mb = W.clone(), b.clone()
+    Z = torch.empty((w.B, w.H, 1, w.d), dtype=torch.float32, device=dev)
+    mb = w.mini_batch
+
+    def step(t, pos0, s):
+        ttt.ttt_linear_decode(t["Q"], t["K"], t["V"], t["eta"], W, b, W_mb, b_mb, gam, bet, pos0=pos0,
+                              mini_batch=mb, ln_eps=w.ln_eps, Z=Z, stream=s)
+
+    # Device rate: one mini-batch cycle of single-token steps (positions 0..b-1)
+    # captured in a CUDA graph, replayed; a decode loop runs this way.
+    stream = torch.cuda.current_stream(dev)
+    for i in range(mb * max(1, -(-args.warmup // mb))):  # whole cycles: the graph starts at position 0
+        step(toks[i % n_tok], i % mb, stream)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream(dev)
+        for i in range(mb):
+            step(toks[i], i, cap)
+    for _ in range(max(1, args.warmup // mb)):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    replays = max(1, -(-args.steps // mb))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(replays):
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    timed_steps = replays * mb
+    total_ms = dist_max(start.elapsed_time(end), world)
+    ms_per_step = total_ms / timed_steps
+    kernel_ms = statistics.mean(a.elapsed_time(c) for a, c in ev) / mb
+    value = w.B * world / (ms_per_step * 1e-3)
+    del graph
+
+    # end to end: each step's token from pinned host memory, z back to the host
+    host_toks = [{k: v.pin_memory() for k, v in
+                  ((k, host[k][:, :, i:i + 1].contiguous()) for k in ("Q", "K", "V", "eta"))}
+                 for i in range(min(n_tok, args.steps))]
+    z_host = torch.empty(Z.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host_toks[0].values())
+    d2h = z_host.numel() * z_host.element_size()
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        t = {k: v.to(dev, non_blocking=True) for k, v in host_toks[i % len(host_toks)].items()}
+        step(t, i % mb, stream)
+        z_host.copy_(Z, non_blocking=True)
+        stream.synchronize()  # the step's z is on the host before the next token is known
+    e2e_s = dist_max((time.perf_counter() - t0) / args.steps, world)
+
+    cpu_base = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_decode_sample(w, host, min(args.ref_seconds, 5.0))
+    if rank == 0:
+        hbm, _, peak_kind = load_peaks()
+        ab = decode_state_bytes(w)
+        achieved = ab / (kernel_ms * 1e-3) / 1e9
+        line = {
+            "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": timed_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(w),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms,
+                         "kernel": "ttt_linear_decode_kernel" if w.d == 64 else "ttt_linear_generic_kernel"},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": w.B * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": timed_steps,
+            "clocks": clk.summary(),
+            "kernel_impl": "decode" if w.d == 64 else "generic",
+            "timing": "CUDA graph of one mini-batch cycle of steps, replayed; e2e: eager calls",
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
     w = WORKLOADS[args.workload]
+    if w.name == "decode_1p3b":
+        return run_decode(args, world, rank, local)
     dev = torch.device("cuda", local)
     host = make_inputs(w, args.seed + rank)
     g = {k: v.to(dev) for k, v in host.items()}
@@ -398,7 +543,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
-                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048])
+                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k == "decode_1p3b"])
     ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split"], default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,

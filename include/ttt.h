@@ -136,6 +136,31 @@ ttt_impl ttt_linear_pick_impl(int B, int H, int T, int d, int mini_batch, ttt_dt
                               ttt_mode mode);
 
 /*
+ * TTT-Linear decode: the scan of ttt_linear_forward continued by T >= 0 more
+ * tokens, the first of them at position pos0 of its mini-batch
+ * (0 <= pos0 < mini_batch, else TTT_ERR_SHAPE).  T = 1 is single-token decode;
+ * T need not fill or end a mini-batch.  The caller keeps the position:
+ * the next call's pos0 is (pos0 + T) % mini_batch.
+ *   W, b       running state W_t, b_t [B][H][d][d], [B][H][d]: read, then
+ *              overwritten with the state after the call's last token
+ *   W_mb, b_mb state the current mini-batch started from, at which its
+ *              gradients are taken: read when pos0 > 0, then overwritten with
+ *              the start state of the mini-batch the next token falls in
+ *              (equal to W, b when the call ends on a mini-batch boundary)
+ *   b, b_mb, ln_gamma, ln_beta may be NULL in TTT_PLAIN.  The four state
+ *   buffers, Z and the inputs must not overlap (TTT_ERR_ALIAS).  Other
+ *   arguments as ttt_linear_forward.  d = 64 runs a decode kernel that keeps
+ *   the state in registers for the whole call (token-serial, fp32); d = 16 and
+ *   32 run the generic fp32 family.  Results equal a ttt_linear_forward over
+ *   the whole stream up to rounding.
+ */
+ttt_status ttt_linear_decode(int B, int H, int T, int d, int mini_batch, int pos0,
+                             ttt_dtype qkv_dtype, ttt_mode mode, float ln_eps, const void* Q,
+                             const void* K, const void* V, const float* eta, float* W, float* b,
+                             float* W_mb, float* b_mb, const float* ln_gamma,
+                             const float* ln_beta, float* Z, ttt_stream_t stream);
+
+/*
  * TTT-MLP forward scan, f(x) = x + LN(GELU(x W1 + b1) W2 + b2).
  *   d = 64 and hidden = 256 are built (TTT_ERR_UNSUPPORTED otherwise).
  *   W1_0 [B][H][d][hidden], b1_0 [B][H][hidden], W2_0 [B][H][hidden][d], b2_0 [B][H][d]

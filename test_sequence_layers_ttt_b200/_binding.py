@@ -57,6 +57,8 @@ lib.ttt_abi_version.restype = _I
 lib.ttt_abi_version.argtypes = []
 lib.ttt_linear_pick_impl.restype = _I
 lib.ttt_linear_pick_impl.argtypes = [_I] * 7
+lib.ttt_linear_decode.restype = _I
+lib.ttt_linear_decode.argtypes = [_I] * 8 + [_F] + [_P] * 11 + [_P]
 
 
 def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
@@ -243,6 +245,37 @@ def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *
         _ptr(b_T), IMPLS[impl], _stream_handle(dev, stream))
     _check(st)
     return rt.to_host((Z, W_T, b_T))
+
+
+def ttt_linear_decode(Q, K, V, eta, W, b, W_mb, b_mb, ln_gamma=None, ln_beta=None, *, pos0: int,
+                      mini_batch: int = 16, mode="ln", ln_eps: float = 1e-6, Z=None, stream=None
+                      ) -> torch.Tensor:
+    """TTT-Linear decode (see include/ttt.h): the scan continued by T tokens from
+    position pos0 of a mini-batch.  W, b (running state) and W_mb, b_mb (the
+    current mini-batch's start state) are CUDA tensors updated in place; the
+    next call's pos0 is (pos0 + T) % mini_batch.  Returns Z."""
+    m = _mode_code(mode)
+    B, H, T, d = Q.shape
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("eta", eta), ("W", W), ("b", b), ("W_mb", W_mb),
+                    ("b_mb", b_mb), ("ln_gamma", ln_gamma), ("ln_beta", ln_beta)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if K.shape != Q.shape or V.shape != Q.shape or K.dtype != Q.dtype or V.dtype != Q.dtype:
+        raise ValueError("Q, K, V must share shape and dtype")
+    if tuple(eta.shape) != (B, H, T) or tuple(W.shape) != (B, H, d, d) or tuple(W_mb.shape) != (B, H, d, d):
+        raise ValueError("eta must be [B,H,T], W and W_mb [B,H,d,d]")
+    for name, t in (("W", W), ("b", b), ("W_mb", W_mb), ("b_mb", b_mb), ("eta", eta)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    dev = Q.device
+    if Z is None:
+        Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    st = lib.ttt_linear_decode(
+        B, H, T, d, int(mini_batch), int(pos0), _dtype_code(Q), m, float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
+        _ptr(eta), _ptr(W), _ptr(b), _ptr(W_mb), _ptr(b_mb), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z),
+        _stream_handle(dev, stream))
+    _check(st)
+    return Z
 
 
 def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,

@@ -83,6 +83,26 @@ ttt_status validate_linear(const LinearArgs& a) {
     return check_aliasing(outs, 3, ins, same_as, 8);
 }
 
+// Decode: the forward scan's checks, plus the position and the mini-batch start
+// state (W_mb, b_mb), which is read and written in place like W and b.
+ttt_status validate_decode(const LinearArgs& a) {
+    ttt_status st = validate_linear(a);
+    if (st != TTT_OK) return st;
+    if (a.pos0 < 0 || a.pos0 >= a.mini_batch) return TTT_ERR_SHAPE;
+    const bool ln = a.mode == TTT_LN_RESIDUAL;
+    if (!a.Wm_T || (ln && !a.bm_T)) return TTT_ERR_NULL;
+    if (!aligned16(a.Wm_T) || (a.bm_T && !aligned16(a.bm_T))) return TTT_ERR_ALIGN;
+    const size_t es = a.dtype == TTT_BF16 ? 2 : 4;
+    const size_t bh = (size_t)a.B * a.H, ntok = bh * (size_t)a.T, d = a.d;
+    const size_t bbytes = ln ? bh * d * 4 : 0;
+    Span ins[] = {{a.Q, ntok * d * es}, {a.K, ntok * d * es}, {a.V, ntok * d * es}, {a.eta, ntok * 4},
+                  {a.gamma, a.gamma ? (size_t)a.H * d * 4 : 0}, {a.beta, a.beta ? (size_t)a.H * d * 4 : 0}};
+    Span outs[] = {{a.Z, ntok * d * 4}, {a.W_T, bh * d * d * 4}, {a.b_T, a.b_T ? bbytes : 0},
+                   {a.Wm_T, bh * d * d * 4}, {a.bm_T, a.bm_T ? bbytes : 0}};
+    const int same_as[] = {-1, -1, -1, -1, -1};
+    return check_aliasing(outs, 5, ins, same_as, 6);
+}
+
 ttt_status validate_mlp(const MlpArgs& a) {
     if (a.B < 1 || a.H < 1 || a.T < 0 || (long long)a.B * a.H > INT_MAX) return TTT_ERR_SHAPE;
     if (!valid_mini_batch(a.mini_batch)) return TTT_ERR_SHAPE;
@@ -161,6 +181,21 @@ static ttt_impl mlp_auto_impl(const MlpArgs& a) {
     return ttt::mlp_generic_supports(a) ? TTT_IMPL_GENERIC : TTT_IMPL_AUTO;
 }
 
+ttt_status ttt_linear_decode(int B, int H, int T, int d, int mini_batch, int pos0, ttt_dtype qkv_dtype,
+                             ttt_mode mode, float ln_eps, const void* Q, const void* K, const void* V,
+                             const float* eta, float* W, float* b, float* W_mb, float* b_mb,
+                             const float* ln_gamma, const float* ln_beta, float* Z, ttt_stream_t stream) {
+    const bool ln = mode == TTT_LN_RESIDUAL;
+    LinearArgs a{B, H, T, d, mini_batch, qkv_dtype, mode, ln_eps, Q, K, V, eta, W, ln ? b : nullptr,
+                 ln_gamma, ln_beta, Z, W, ln ? b : nullptr,
+                 pos0, pos0 > 0 ? W_mb : nullptr, (pos0 > 0 && ln) ? b_mb : nullptr, W_mb, ln ? b_mb : nullptr};
+    ttt_status st = validate_decode(a);
+    if (st != TTT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (ttt::linear_decode_supports(a)) return finish(ttt::launch_linear_decode(a, s), s);
+    return finish(ttt::launch_linear_generic(a, s), s);
+}
+
 ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                                 ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
                                 const void* V, const float* eta, const float* W1_0, const float* b1_0,
@@ -220,6 +255,6 @@ const char* ttt_status_string(ttt_status status) {
     }
 }
 
-int ttt_abi_version(void) { return 100; }
+int ttt_abi_version(void) { return 101; }
 
 }  // extern "C"

@@ -15,6 +15,11 @@ struct LinearArgs {
     const void *Q, *K, *V;
     const float *eta, *W0, *b0, *gamma, *beta;
     float *Z, *W_T, *b_T;
+    // decode only (generic family): position of the first token in its
+    // mini-batch, and the mini-batch start state in (read when pos0 > 0) and out
+    int pos0;
+    const float *Wm0, *bm0;
+    float *Wm_T, *bm_T;
 };
 
 struct MlpArgs {
@@ -31,6 +36,10 @@ cudaError_t launch_linear_generic(const LinearArgs& a, cudaStream_t stream);
 
 bool linear_tc_supports(const LinearArgs& a);
 cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream);
+
+// Decode with the state in registers (d = 64); in place on W_T / b_T and Wm_T / bm_T.
+bool linear_decode_supports(const LinearArgs& a);
+cudaError_t launch_linear_decode(const LinearArgs& a, cudaStream_t stream);
 
 bool mlp_generic_supports(const MlpArgs& a);
 cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);

@@ -16,6 +16,14 @@
 //   z      = q + LN(zbar)           (plain mode: z = zbar)
 //   W_c   -= K^T diag(eta) G,  b_c -= eta^T G
 // and W_s := W_c at every mini-batch boundary.
+//
+// Decode (the scan continued by T tokens from position pos0 of a mini-batch)
+// runs the same loop with the chunks aligned to the stream's mini-batches
+// rather than to the call's first token: a chunk never crosses a mini-batch
+// boundary, W_s comes in with the call when pos0 > 0, and goes out as the
+// start state of the mini-batch the next token falls in.
+#include <atomic>
+
 #include "common.cuh"
 #include "ttt_internal.h"
 
@@ -45,7 +53,8 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
                           const Tin* __restrict__ K, const Tin* __restrict__ V,
                           const float* __restrict__ eta, const float* W0, const float* b0,
                           const float* __restrict__ gamma, const float* __restrict__ beta,
-                          float* __restrict__ Z, float* W_T, float* b_T) {
+                          float* __restrict__ Z, float* W_T, float* b_T, int pos0, const float* Ws0,
+                          const float* bs0, float* Ws_T, float* bs_T) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     LinearSmem<D>& s = *reinterpret_cast<LinearSmem<D>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -54,17 +63,21 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
     const int C = mb < kChunk ? mb : kChunk;
 
     for (int i = tid; i < D * D; i += kThreads) s.Wc[i] = W0[bh * D * D + i];
+    if (Ws0 != nullptr)  // decode from inside a mini-batch: its start state comes with the call
+        for (int i = tid; i < D * D; i += kThreads) s.Ws[i] = Ws0[bh * D * D + i];
     for (int j = tid; j < D; j += kThreads) {
+        s.bs[j] = (kPlain || bs0 == nullptr) ? 0.f : bs0[bh * D + j];
         s.bc[j] = (kPlain || b0 == nullptr) ? 0.f : b0[bh * D + j];
         s.gam[j] = kPlain ? 1.f : gamma[(long)h * D + j];
         s.bet[j] = kPlain ? 0.f : beta[(long)h * D + j];
     }
 
     const long tok0 = bh * (long)T;
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int n = min(C, T - t0);
+    for (int t0 = 0, n = 0; t0 < T; t0 += n) {
+        const int ph = (pos0 + t0) % mb;  // position of the chunk's first token in its mini-batch
+        n = min(min(C, T - t0), mb - ph);
         __syncthreads();  // previous chunk fully consumed
-        if (t0 % mb == 0) {  // mini-batch boundary: W_s := W_c
+        if (ph == 0) {  // mini-batch boundary: W_s := W_c
             for (int i = tid; i < D * D; i += kThreads) s.Ws[i] = s.Wc[i];
             for (int j = tid; j < D; j += kThreads) s.bs[j] = s.bc[j];
         }
@@ -79,8 +92,8 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
         for (int t = tid; t < C; t += kThreads) s.eta[t] = t < n ? eta[tok0 + t0 + t] : 0.f;
         __syncthreads();
 
-        // y = X W_s (+ b_s), ZQ = Q W_c (+ b_c), A
-        for (int o = tid; o < C * D; o += kThreads) {
+        // y = X W_s (+ b_s), ZQ = Q W_c (+ b_c), A; only the chunk's n tokens
+        for (int o = tid; o < n * D; o += kThreads) {
             int t = o / D, j = o % D;
             float y = kPlain ? 0.f : s.bs[j];
             float zq = kPlain ? 0.f : s.bc[j];
@@ -97,7 +110,7 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
         for (int o = tid; o < C * C; o += kThreads) {
             int t = o / C, u = o % C;
             float a = 0.f;
-            if (u <= t) {
+            if (u <= t && t < n) {
                 float dot = 0.f;
                 for (int i = 0; i < D; i++) dot = fmaf(s.Qt[t * D + i], s.X[u * D + i], dot);
                 a = s.eta[u] * (kPlain ? dot : dot + 1.f);
@@ -107,7 +120,7 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
         __syncthreads();
 
         // G = dl/dy, one warp per token
-        for (int t = warp; t < C; t += kThreads / 32) {
+        for (int t = warp; t < n; t += kThreads / 32) {
             float* y = s.Y + t * D;
             if (kPlain) {
                 for (int j = lane; j < D; j += 32) y[j] = 2.f * (y[j] - s.Vt[t * D + j]);
@@ -143,7 +156,7 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
         __syncthreads();
 
         // zbar = ZQ - A G ; state update W_c -= X^T diag(eta) G, b_c -= eta^T G
-        for (int o = tid; o < C * D; o += kThreads) {
+        for (int o = tid; o < n * D; o += kThreads) {
             int t = o / D, j = o % D;
             float z = s.ZQ[o];
             for (int u = 0; u <= t; u++) z = fmaf(-s.A[t * C + u], s.Y[u * D + j], z);
@@ -152,13 +165,13 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
         for (int o = tid; o < D * D; o += kThreads) {
             int i = o / D, j = o % D;
             float acc = 0.f;
-            for (int u = 0; u < C; u++) acc = fmaf(s.X[u * D + i] * s.eta[u], s.Y[u * D + j], acc);
+            for (int u = 0; u < n; u++) acc = fmaf(s.X[u * D + i] * s.eta[u], s.Y[u * D + j], acc);
             s.Wc[o] -= acc;
         }
         if (!kPlain)
             for (int j = tid; j < D; j += kThreads) {
                 float acc = 0.f;
-                for (int u = 0; u < C; u++) acc = fmaf(s.eta[u], s.Y[u * D + j], acc);
+                for (int u = 0; u < n; u++) acc = fmaf(s.eta[u], s.Y[u * D + j], acc);
                 s.bc[j] -= acc;
             }
         __syncthreads();
@@ -185,17 +198,35 @@ ttt_linear_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict
     for (int i = tid; i < D * D; i += kThreads) W_T[bh * D * D + i] = s.Wc[i];
     if (!kPlain && b_T != nullptr)
         for (int j = tid; j < D; j += kThreads) b_T[bh * D + j] = s.bc[j];
+    if (Ws_T != nullptr) {
+        // start state of the mini-batch the next token falls in
+        const bool boundary = (pos0 + T) % mb == 0;
+        for (int i = tid; i < D * D; i += kThreads) Ws_T[bh * D * D + i] = boundary ? s.Wc[i] : s.Ws[i];
+        if (!kPlain && bs_T != nullptr)
+            for (int j = tid; j < D; j += kThreads) bs_T[bh * D + j] = boundary ? s.bc[j] : s.bs[j];
+    }
 }
 
 template <int D, typename Tin, bool kPlain>
 cudaError_t launch_one(const LinearArgs& a, cudaStream_t stream) {
     auto kern = ttt_linear_generic_kernel<D, Tin, kPlain>;
     const size_t smem = sizeof(LinearSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // the shared-memory limit is set once per device, so that a launch (a
+    // decode step, say, captured in a CUDA graph) makes no other runtime call
+    static std::atomic<unsigned long long> attr_set{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit);
+    }
     kern<<<a.B * a.H, kThreads, smem, stream>>>(
         a.H, a.T, a.mini_batch, a.ln_eps, static_cast<const Tin*>(a.Q), static_cast<const Tin*>(a.K),
-        static_cast<const Tin*>(a.V), a.eta, a.W0, a.b0, a.gamma, a.beta, a.Z, a.W_T, a.b_T);
+        static_cast<const Tin*>(a.V), a.eta, a.W0, a.b0, a.gamma, a.beta, a.Z, a.W_T, a.b_T, a.pos0, a.Wm0,
+        a.bm0, a.Wm_T, a.bm_T);
     return cudaPeekAtLastError();
 }
 

@@ -61,6 +61,9 @@ WORKLOADS: Dict[str, Workload] = {
     "linear_125m_2k": Workload("linear_125m_2k", "linear", 8, 12, 2048, 64, 16, "bf16", init="lm"),
     # 1.3B-class TTT-Linear layer, 32k context: B=2, H=32, d=64, T=32768, b=16.
     "linear_1p3b_32k": Workload("linear_1p3b_32k", "linear", 2, 32, 32768, 64, 16, "bf16", init="lm"),
+    # Decode on the 1.3B-class layer: the stream of B=2 sequences x H=32 heads
+    # continued one token per step; T is the number of tokens generated.
+    "decode_1p3b": Workload("decode_1p3b", "linear", 2, 32, 256, 64, 16, "bf16", init="lm"),
     # TTT-MLP layer: B=4, H=12, d=64, 64 -> 256 -> 64, T=8192, b=16.
     "mlp_8k": Workload("mlp_8k", "mlp", 4, 12, 8192, 64, 16, "bf16", hidden=256, init="mlp"),
 }

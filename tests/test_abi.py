@@ -45,7 +45,7 @@ def test_status_strings():
     for code, name in enumerate(b.STATUS):
         assert b.status_string(code).startswith(name)
     assert b.status_string(99) == "TTT_ERR_UNKNOWN"
-    assert b.lib.ttt_abi_version() == 100
+    assert b.lib.ttt_abi_version() == 101
 
 
 # Fake, 16-byte aligned, non-overlapping device addresses.  Never dereferenced:
@@ -137,6 +137,38 @@ def test_mlp_alias_and_align():
     p[10] = p[2] + 1024  # Z inside V
     assert mlp_call(ptrs=p) == ALIAS
     assert mlp_call(ptrs=with_ptr(13, fake(13) + 4, 15)) == ALIGN
+
+
+# decode: Q K V eta W b W_mb b_mb gamma beta Z
+def decode_call(B=1, H=2, T=64, d=64, mb=16, pos0=0, dtype=0, mode=0, eps=1e-6, ptrs=None):
+    p = [fake(i) for i in range(11)] if ptrs is None else ptrs
+    return b.lib.ttt_linear_decode(B, H, T, d, mb, pos0, dtype, mode, eps, *p, None)
+
+
+@pytest.mark.parametrize("pos0", [-1, 16, 100])
+def test_decode_position_outside_the_mini_batch(pos0):
+    assert decode_call(pos0=pos0) == SHAPE
+
+
+def test_decode_bad_mini_batch():
+    assert decode_call(mb=12) == SHAPE
+
+
+@pytest.mark.parametrize("idx", [4, 6, 7, 8, 9])
+def test_decode_null_state_or_ln_params(idx):
+    assert decode_call(ptrs=with_ptr(idx, None)) == NULL
+
+
+@pytest.mark.parametrize("idx", [4, 5, 6, 7, 10])
+def test_decode_misaligned_state_or_output(idx):
+    assert decode_call(ptrs=with_ptr(idx, fake(idx) + 4)) == ALIGN
+
+
+@pytest.mark.parametrize("dst,src,off", [(6, 4, 64), (6, 10, 0), (7, 0, 128), (4, 6, 16), (10, 5, 0)])
+def test_decode_overlapping_buffers(dst, src, off):
+    p = [fake(k) for k in range(11)]
+    p[dst] = p[src] + off
+    assert decode_call(ptrs=p) == ALIAS
 
 
 def test_linear_has_no_split_family():

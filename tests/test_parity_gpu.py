@@ -264,6 +264,141 @@ def test_linear_host_pipeline_uneven_groups(ttt, mode):
         np.testing.assert_array_equal(host[2].numpy(), dev[2])
 
 
+# ------------------------------------------------------------------ TTT-Linear decode
+
+def gpu_decode_pieces(ttt, w, inp, cuts, mini_batch=None):
+    """Decode calls over [0, T) cut at `cuts`, the state carried on the GPU."""
+    mb = mini_batch or w.mini_batch
+    g = to_cuda(inp)
+    plain = w.mode == MODE_PLAIN
+    W = g["W0"].clone()
+    b = None if plain else g["b0"].clone()
+    W_mb = torch.zeros_like(W)
+    b_mb = None if plain else torch.zeros_like(b)
+    T = g["Q"].shape[2]
+    bounds = [0, *cuts, T]
+    Zs = []
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = lambda x: x[:, :, a:c].contiguous()
+        Zs.append(ttt.ttt_linear_decode(sl(g["Q"]), sl(g["K"]), sl(g["V"]), sl(g["eta"]), W, b, W_mb, b_mb,
+                                        None if plain else g["gamma"], None if plain else g["beta"],
+                                        pos0=a % mb, mini_batch=mb, mode="plain" if plain else "ln",
+                                        ln_eps=w.ln_eps))
+    torch.cuda.synchronize()
+    out = [torch.cat(Zs, dim=2), W, b, W_mb, b_mb]
+    return [None if o is None else o.cpu().numpy() for o in out]
+
+
+def oracle_decode_pieces(w, inp, cuts, mini_batch=None):
+    mb = mini_batch or w.mini_batch
+    T = inp["Q"].shape[2]
+    W, b, W_mb, b_mb = inp["W0"], inp["b0"], None, None
+    bounds = [0, *cuts, T]
+    Zs = []
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = lambda x: x[:, :, a:c]
+        Z, W, b, W_mb, b_mb = oracle.ttt_linear_decode(sl(inp["Q"]), sl(inp["K"]), sl(inp["V"]),
+                                                       sl(inp["eta"]), W, b, W_mb, b_mb, inp["gamma"],
+                                                       inp["beta"], mb, a % mb, w.mode, w.ln_eps)
+        Zs.append(Z)
+    return [np.concatenate(Zs, axis=2), W, b, W_mb, b_mb]
+
+
+def compare_decode(out, ref, f, plain):
+    assert_close(out[0], ref[0], f, "Z")
+    for name, i in (("W", 1), ("W_mb", 3)):
+        assert_close(out[i], ref[i], f, name)
+    if not plain:
+        for name, i in (("b", 2), ("b_mb", 4)):
+            assert_close(out[i], ref[i], f, name, denom=max(rms(ref[i]), rms(ref[1])))
+
+
+@pytest.mark.parametrize("name,shape,mb,cuts", [
+    ("linear_125m_2k", dict(B=1, H=2, T=96), 16, [5, 6, 21, 40, 64, 79]),
+    ("linear_125m_2k", dict(B=2, H=3, T=100), 32, [1, 33, 50]),
+    ("linear_tiny_f32", {}, 16, [3, 17, 18, 47]),
+    ("linear_tiny_f32", {}, 8, [1, 2, 3, 12, 29]),
+    ("theorem1_f32", dict(B=1, H=2, T=80), 80, [7, 30, 31]),
+    ("linear_125m_2k", dict(B=1, H=2, T=24), 1, [5, 9]),          # b = 1: online GD
+    ("linear_125m_2k", dict(B=1, H=2, T=48, d=32), 16, [5, 21]),  # d = 32: generic family
+])
+def test_linear_decode_pieces_vs_oracle(ttt, name, shape, mb, cuts):
+    """Decode calls cut anywhere (inside mini-batches, ragged tails) against the
+    oracle's decode over the same pieces."""
+    w = WORKLOADS[name].with_shape(**shape) if shape else WORKLOADS[name]
+    inp = make_inputs(w, 2)
+    out = gpu_decode_pieces(ttt, w, inp, cuts, mb)
+    ref = oracle_decode_pieces(w, inp, cuts, mb)
+    compare_decode(out, ref, TOL[w.dtype], w.mode == MODE_PLAIN)
+
+
+def test_linear_decode_token_by_token_equals_forward_oracle(ttt):
+    """Single-token decode steps over a stream reproduce the oracle's forward scan."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=40)
+    inp = make_inputs(w, 3)
+    out = gpu_decode_pieces(ttt, w, inp, list(range(1, 40)))
+    Zo, Wo, bo = oracle_linear(w, inp)
+    f = TOL[w.dtype]
+    assert_close(out[0], Zo, f, "Z")
+    assert_close(out[1], Wo, f, "W")
+    assert_close(out[2], bo, f, "b", denom=max(rms(bo), rms(Wo)))
+
+
+def test_linear_decode_one_call_is_the_generic_forward(ttt):
+    """From a mini-batch boundary, one decode call at d = 32 (generic family)
+    runs the generic forward scan operation for operation."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=2, T=72, d=32)
+    inp = make_inputs(w, 4)
+    dec = gpu_decode_pieces(ttt, w, inp, [])
+    fwd = gpu_linear(ttt, w, inp, impl="generic")
+    np.testing.assert_array_equal(dec[0], fwd[0])
+    np.testing.assert_array_equal(dec[1], fwd[1])
+    np.testing.assert_array_equal(dec[2], fwd[2])
+    # 72 = 4 * 16 + 8 tokens: the call ends inside a mini-batch, whose start
+    # state is the state after 64 tokens
+    first = {k: (v[:, :, :64].contiguous() if k in ("Q", "K", "V", "eta") else v) for k, v in inp.items()}
+    fwd64 = gpu_linear(ttt, w.with_shape(T=64), first, impl="generic")
+    np.testing.assert_array_equal(dec[3], fwd64[1])
+    np.testing.assert_array_equal(dec[4], fwd64[2])
+
+
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_linear_decode_register_kernel_matches_generic_forward(ttt, mode):
+    """d = 64 decode (state in registers, token-serial) against the generic
+    forward scan: the same fp32 arithmetic in another order."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=2, T=72, mode=MODE_PLAIN if mode == "plain" else 0)
+    inp = make_inputs(w, 6)
+    dec = gpu_decode_pieces(ttt, w, inp, [])
+    fwd = gpu_linear(ttt, w, inp, impl="generic")
+    assert_close(dec[0], fwd[0].astype(np.float64), 1e-4, "Z")
+    assert_close(dec[1], fwd[1].astype(np.float64), 1e-4, "W")
+    if mode == "ln":
+        assert_close(dec[2], fwd[2].astype(np.float64), 1e-4, "b", denom=max(rms(fwd[2]), rms(fwd[1])))
+
+
+def test_linear_decode_empty_call_keeps_state(ttt):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=0)
+    g = to_cuda(make_inputs(w, 5))
+    W, b = g["W0"].clone(), g["b0"].clone()
+    W_mb, b_mb = W + 0.5, b - 0.5
+    W_mb0, b_mb0 = W_mb.clone(), b_mb.clone()
+    Z = ttt.ttt_linear_decode(g["Q"], g["K"], g["V"], g["eta"], W, b, W_mb, b_mb, g["gamma"], g["beta"],
+                              pos0=5, mini_batch=16)
+    torch.cuda.synchronize()
+    assert Z.shape == (1, 2, 0, 64)
+    assert torch.equal(W, g["W0"]) and torch.equal(W_mb, W_mb0) and torch.equal(b_mb, b_mb0)
+
+
+def test_linear_decode_bad_position(ttt):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=1, T=4)
+    g = to_cuda(make_inputs(w, 0))
+    W, b = g["W0"].clone(), g["b0"].clone()
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_linear_decode(g["Q"], g["K"], g["V"], g["eta"], W, b, W.clone(), b.clone(), g["gamma"],
+                              g["beta"], pos0=16, mini_batch=16)
+    assert ei.value.status == 2
+
+
 # ------------------------------------------------------------------ TTT-MLP
 
 # the tensor-core families: one CTA per scan, and each scan's hidden units
