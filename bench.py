@@ -404,7 +404,9 @@ def run_decode(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": workload_config(w),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / hbm,
+                         "traffic": recorded_traffic("ttt_linear_decode_kernel", w.name) if w.d == 64 else None,
+                         "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms,
                          "kernel": "ttt_linear_decode_kernel" if w.d == 64 else "ttt_linear_generic_kernel"},
             "cpu_baseline": cpu_base,
