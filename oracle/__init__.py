@@ -48,6 +48,9 @@ def _load():
             f = getattr(lib, "oracle_ttt_mlp" + sfx)
             f.restype = I
             f.argtypes = [I, I, I, I, I, I, real] + [P] * 15 + [I]
+            f = getattr(lib, "oracle_ttt_mlp_decode" + sfx)
+            f.restype = I
+            f.argtypes = [I, I, I, I, I, I, I, real] + [P] * 15 + [I]
             f = getattr(lib, "oracle_linear_loss_grad" + sfx)
             f.restype = real
             f.argtypes = [I, I, real] + [P] * 8
@@ -145,6 +148,32 @@ def ttt_mlp(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, gamma, beta, mini_batch: int,
     if rc != 0:
         raise ValueError("oracle_ttt_mlp: bad arguments")
     return Z, W1_T, b1_T, W2_T, b2_T
+
+
+def ttt_mlp_decode(Q, K, V, eta, W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb, gamma, beta,
+                   mini_batch: int, pos0: int, ln_eps: float = 1e-6, precision: str = "f64",
+                   threads: Optional[int] = None):
+    """TTT-MLP scan continued by T tokens from position pos0 of a mini-batch.
+
+    (W1, b1, W2, b2): running state; (W1_mb, ...): the state the current
+    mini-batch started from (read when pos0 > 0; None means a copy of the
+    running state).  Returns (Z, W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb)
+    after the T tokens.  The inputs are not modified."""
+    dt = np.float64 if precision == "f64" else np.float32
+    Q, K, V, eta = (_arr(x, dt) for x in (Q, K, V, eta))
+    B, H, T, d = Q.shape
+    run = [_arr(x, dt).copy() for x in (W1, b1, W2, b2)]
+    start = [(_arr(x, dt).copy() if x is not None else r.copy()) for x, r in zip((W1_mb, b1_mb, W2_mb, b2_mb), run)]
+    gamma, beta = _arr(gamma, dt), _arr(beta, dt)
+    hid = run[0].shape[-1]
+    Z = np.zeros((B, H, T, d), dt)
+    fn = getattr(_load(), "oracle_ttt_mlp_decode_" + precision)
+    rc = fn(B, H, T, d, hid, int(mini_batch), int(pos0), ln_eps, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta),
+            *(_ptr(x) for x in run), *(_ptr(x) for x in start), _ptr(gamma), _ptr(beta), _ptr(Z),
+            _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle_ttt_mlp_decode: bad arguments")
+    return (Z, *run, *start)
 
 
 def linear_loss_grad(k, v, W, b, gamma, beta, mode: int = MODE_LN_RESIDUAL,

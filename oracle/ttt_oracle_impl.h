@@ -394,6 +394,67 @@ int FN(oracle_ttt_mlp)(int B, int H, int T, int d, int hid, int mb, REAL eps, co
     return 0;
 }
 
+/*
+ * TTT-MLP decode: the MLP scan continued by T tokens from position pos0 of a
+ * mini-batch, as oracle_ttt_linear_decode for the linear model [LR1], [LR5],
+ * [ABS].  (W1c, b1c, W2c, b2c) is the running state, (W1m, b1m, W2m, b2m)
+ * the state the current mini-batch started from; all are read and
+ * overwritten in place.  Returns 0, or -1 on bad arguments.
+ */
+int FN(oracle_ttt_mlp_decode)(int B, int H, int T, int d, int hid, int mb, int pos0, REAL eps,
+                              const REAL* Q, const REAL* K, const REAL* V, const REAL* eta,
+                              REAL* W1c_all, REAL* b1c_all, REAL* W2c_all, REAL* b2c_all,
+                              REAL* W1m_all, REAL* b1m_all, REAL* W2m_all, REAL* b2m_all,
+                              const REAL* gamma, const REAL* beta, REAL* Z, int nthreads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || hid <= 0 || mb <= 0 || pos0 < 0 || pos0 >= mb) return -1;
+    if (nthreads <= 0) nthreads = 1;
+    long nbh = (long)B * H;
+    size_t nW = (size_t)d * hid;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < nbh; bh++) {
+        int h = (int)(bh % H);
+        const REAL* gam = gamma + (long)h * d;
+        const REAL* bet = beta + (long)h * d;
+        REAL *W1c = W1c_all + bh * nW, *W2c = W2c_all + bh * nW, *b1c = b1c_all + bh * hid, *b2c = b2c_all + bh * d;
+        REAL *W1m = W1m_all + bh * nW, *W2m = W2m_all + bh * nW, *b1m = b1m_all + bh * hid, *b2m = b2m_all + bh * d;
+        REAL* vec = (REAL*)malloc(sizeof(REAL) * (size_t)(2 * hid + 5 * d + hid));
+        REAL *a = vec, *g1 = vec + hid, *g2 = vec + 2 * hid, *scratch = g2 + d;
+        for (int t = 0; t < T; t++) {
+            if ((pos0 + t) % mb == 0) { /* a mini-batch starts at this token */
+                memcpy(W1m, W1c, sizeof(REAL) * nW);
+                memcpy(W2m, W2c, sizeof(REAL) * nW);
+                memcpy(b1m, b1c, sizeof(REAL) * hid);
+                memcpy(b2m, b2c, sizeof(REAL) * d);
+            }
+            long row = (bh * T + t) * d;
+            REAL e = eta[bh * T + t];
+            FN(mlp_token_grads)(d, hid, eps, K + row, V + row, W1m, b1m, W2m, b2m, gam, bet, a, g1, g2,
+                                scratch);
+            for (int i = 0; i < d; i++) {
+                REAL ek = e * K[row + i];
+                REAL* W1i = W1c + (long)i * hid;
+                for (int j = 0; j < hid; j++) W1i[j] -= ek * g1[j];
+            }
+            for (int j = 0; j < hid; j++) b1c[j] -= e * g1[j];
+            for (int i = 0; i < hid; i++) {
+                REAL ea = e * a[i];
+                REAL* W2i = W2c + (long)i * d;
+                for (int j = 0; j < d; j++) W2i[j] -= ea * g2[j];
+            }
+            for (int j = 0; j < d; j++) b2c[j] -= e * g2[j];
+            FN(mlp_apply)(d, hid, eps, Q + row, W1c, b1c, W2c, b2c, gam, bet, Z + row, scratch);
+        }
+        if ((pos0 + T) % mb == 0) { /* the next token starts a mini-batch */
+            memcpy(W1m, W1c, sizeof(REAL) * nW);
+            memcpy(W2m, W2c, sizeof(REAL) * nW);
+            memcpy(b1m, b1c, sizeof(REAL) * hid);
+            memcpy(b2m, b2c, sizeof(REAL) * d);
+        }
+        free(vec);
+    }
+    return 0;
+}
+
 #undef FN
 #undef CAT
 #undef CAT_

@@ -540,6 +540,37 @@ def test_decode_rejects_bad_position(pos0):
         oracle.ttt_linear_decode(Q, K, V, eta, W0, b0, W0, b0, gamma, beta, 16, pos0)
 
 
+@pytest.mark.parametrize("mb,cuts", [(8, [1, 2, 3, 13, 21]), (16, [5, 6, 21]), (1, [4, 9]), (32, [7, 30])])
+def test_mlp_decode_pieces_equal_minibatch_rule(mb, cuts):
+    """TTT-MLP decode calls cut anywhere reproduce the mini-batch rule written out
+    with torch autograd over the whole stream."""
+    Q, K, V, eta, W1, b1, W2, b2, gamma, beta = small_mlp_case(5, T=32)
+    T = Q.shape[2]
+    state = [W1, b1, W2, b2]
+    start = [None] * 4
+    Zs = []
+    bounds = [0, *cuts, T]
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = (slice(None), slice(None), slice(a, c))
+        out = oracle.ttt_mlp_decode(Q[sl], K[sl], V[sl], eta[sl], *state, *start, gamma, beta, mb, a % mb)
+        Zs.append(out[0])
+        state, start = list(out[1:5]), list(out[5:9])
+    fn = (lambda x, W1_, b1_, W2_, b2_: f_mlp(x, W1_, b1_, W2_, b2_, t64(gamma[0]), t64(beta[0])))
+    Zr, params = minibatch_restatement(fn, [t64(p[0, 0]) for p in (W1, b1, W2, b2)], t64(Q[0, 0]),
+                                       t64(K[0, 0]), t64(V[0, 0]), t64(eta[0, 0]), mb)
+    assert rel(np.concatenate(Zs, axis=2)[0, 0], Zr.numpy()) < 1e-11
+    for got, ref in zip(state, params):
+        assert rel(got[0, 0], ref.numpy()) < 1e-11
+
+
+def test_mlp_decode_whole_stream_is_the_forward_scan():
+    Q, K, V, eta, W1, b1, W2, b2, gamma, beta = small_mlp_case(6, T=40)
+    dec = oracle.ttt_mlp_decode(Q, K, V, eta, W1, b1, W2, b2, None, None, None, None, gamma, beta, 16, 0)
+    fwd = oracle.ttt_mlp(Q, K, V, eta, W1, b1, W2, b2, gamma, beta, 16)
+    for a, b in zip(dec[:5], fwd):
+        np.testing.assert_array_equal(a, b)
+
+
 MUTATIONS = {
     "drop_mean_term": ("g[j] = s * (g[j] - mean_gx - xhat[j] * mean_gxx);",
                        "g[j] = s * (g[j] - xhat[j] * mean_gxx);"),
@@ -563,6 +594,9 @@ MUTATIONS = {
     "decode_gradient_at_running_state": (
         "FN(linear_token_dy)(d, mode, eps, K + row, V + row, Wm, bm, gam, bet, g, scratch);",
         "FN(linear_token_dy)(d, mode, eps, K + row, V + row, Wc, bc, gam, bet, g, scratch);"),
+    "mlp_decode_gradient_at_running_state": (
+        "FN(mlp_token_grads)(d, hid, eps, K + row, V + row, W1m, b1m, W2m, b2m, gam, bet, a, g1, g2,",
+        "FN(mlp_token_grads)(d, hid, eps, K + row, V + row, W1c, b1c, W2c, b2c, gam, bet, a, g1, g2,"),
     "decode_no_minibatch_restart": (
         "if ((pos0 + t) % mb == 0) { /* a mini-batch starts at this token */",
         "if (0) {"),
@@ -616,6 +650,7 @@ def _run_pins_with(lib_path):
         lambda: test_minibatch_rule_mlp(8, 24),
         lambda: test_decode_pieces_equal_minibatch_rule(LN, 8, [1, 2, 3, 19, 33]),
         test_decode_single_tokens_theorem1,
+        lambda: test_mlp_decode_pieces_equal_minibatch_rule(8, [1, 2, 3, 13, 21]),
     ]
     try:
         for pin in pins:
