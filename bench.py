@@ -42,6 +42,8 @@ def metric_name(w) -> str:
         return METRIC
     if w.name == "decode_1p3b":
         return "TTT-Linear decode tokens/sec on 1 B200 (1.3B-layer shape, one token per sequence per step)"
+    if w.name == "decode_mlp_8k":
+        return "TTT-MLP decode tokens/sec on 1 B200 (TTT-MLP layer shape, one token per sequence per step)"
     shape = {"linear_125m_2k": "125M-layer shape, 2k ctx", "mlp_8k": "TTT-MLP layer, 8k ctx"}[w.name]
     return f"TTT forward tokens/sec on 1 B200 ({shape}); % of roofline"
 FALLBACK_HBM_GBS = 6650.0
@@ -240,11 +242,17 @@ def cpu_oracle_sample(w, inp, target_s: float):
                       f"{dt:.2f} s; tokens counted as scans*T/H"}
 
 
+DECODE_WORKLOADS = ("decode_1p3b", "decode_mlp_8k")
+
+
 def decode_state_bytes(w) -> int:
     """Algorithmic bytes of one decode step (one token for every (batch, head)
-    stream): running state W, b read and written, the mini-batch start state
-    W_mb, b_mb read and written, and the token's q, k, v, eta in and z out."""
-    state = 4 * (w.d * w.d + w.d)
+    stream): running state read and written, the mini-batch start state read
+    and written, and the token's q, k, v, eta in and z out."""
+    if w.kind == "mlp":
+        state = 4 * (2 * w.d * w.hidden + w.hidden + w.d)
+    else:
+        state = 4 * (w.d * w.d + w.d)
     es = 2 if w.dtype == "bf16" else 4
     return w.B * w.H * (4 * state + 3 * w.d * es + 4 + w.d * 4)
 
@@ -255,14 +263,22 @@ def cpu_oracle_decode_sample(w, inp, target_s: float):
     counts one token per sequence per step (B per step)."""
     import oracle
     cores = os.cpu_count() or 1
-    W, b, W_mb, b_mb = inp["W0"], inp["b0"], None, None
+    if w.kind == "mlp":
+        run, start = [inp[k] for k in ("W1_0", "b1_0", "W2_0", "b2_0")], [None] * 4
+    else:
+        W, b, W_mb, b_mb = inp["W0"], inp["b0"], None, None
     steps, t0 = 0, time.perf_counter()
     while True:
         i = steps % w.T
         sl = {k: inp[k][:, :, i:i + 1] for k in ("Q", "K", "V", "eta")}
-        _, W, b, W_mb, b_mb = oracle.ttt_linear_decode(sl["Q"], sl["K"], sl["V"], sl["eta"], W, b, W_mb, b_mb,
-                                                       inp["gamma"], inp["beta"], w.mini_batch,
-                                                       i % w.mini_batch, w.mode, w.ln_eps, threads=cores)
+        if w.kind == "mlp":
+            out = oracle.ttt_mlp_decode(sl["Q"], sl["K"], sl["V"], sl["eta"], *run, *start, inp["gamma"],
+                                        inp["beta"], w.mini_batch, i % w.mini_batch, w.ln_eps, threads=cores)
+            run, start = list(out[1:5]), list(out[5:9])
+        else:
+            _, W, b, W_mb, b_mb = oracle.ttt_linear_decode(sl["Q"], sl["K"], sl["V"], sl["eta"], W, b, W_mb, b_mb,
+                                                           inp["gamma"], inp["beta"], w.mini_batch,
+                                                           i % w.mini_batch, w.mode, w.ln_eps, threads=cores)
         steps += 1
         dt = time.perf_counter() - t0
         if dt >= target_s:
@@ -277,7 +293,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     inp = make_inputs(w, args.seed)
-    sample = cpu_oracle_decode_sample if args.workload == "decode_1p3b" else cpu_oracle_sample
+    sample = cpu_oracle_decode_sample if args.workload in DECODE_WORKLOADS else cpu_oracle_sample
     for _ in range(args.warmup):
         sample(w, inp, 0.5)
     vals, samples = [], None
@@ -304,12 +320,15 @@ def run_reference(args, world, rank):
 
 
 def workload_config(w):
-    if w.name == "decode_1p3b":
+    if w.name in DECODE_WORKLOADS:
+        mb_state = 4 * w.B * w.H * 2 * ((2 * w.d * w.hidden + w.hidden + w.d) if w.kind == "mlp" else (w.d * w.d + w.d))
         return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "mini_batch": w.mini_batch,
-                "qkv_dtype": w.dtype, "state_dtype": "f32", "inner_model": "x + LN(xW + b)",
+                "qkv_dtype": w.dtype, "state_dtype": "f32",
+                "inner_model": (f"x + LN(MLP {w.d}->{w.hidden}->{w.d}, GELU)" if w.kind == "mlp"
+                                else "x + LN(xW + b)"),
                 "step": "one token for each of the B x H streams; positions cycle through the mini-batch",
                 "timed": "steps rounded up to whole mini-batch cycles",
-                "l2": "no flush: the 4.3 MB state stays in L2 between steps, as in a decode loop"}
+                "l2": f"no flush: the {mb_state / 1e6:.1f} MB state stays in L2 between steps, as in a decode loop"}
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "mini_batch": w.mini_batch,
             "qkv_dtype": w.dtype, "state_dtype": "f32",
             "inner_model": (f"x + LN(MLP {w.d}->{w.hidden}->{w.d}, GELU)" if w.kind == "mlp"
@@ -319,7 +338,7 @@ def workload_config(w):
 
 def run_decode(args, world, rank, local):
     """Single-token decode steps through ttt_linear_decode (d = 64: the decode
-    kernel with the state in registers)."""
+    kernel with the state in registers) or ttt_mlp_decode (generic family)."""
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
     w = WORKLOADS[args.workload]
@@ -329,14 +348,22 @@ def run_decode(args, world, rank, local):
     toks = [{k: host[k][:, :, i:i + 1].contiguous().to(dev) for k in ("Q", "K", "V", "eta")}
             for i in range(n_tok)]
     gam, bet = host["gamma"].to(dev), host["beta"].to(dev)
-    W, b = host["W0"].to(dev), host["b0"].to(dev)
-    W_mb, b_mb = W.clone(), b.clone()
     Z = torch.empty((w.B, w.H, 1, w.d), dtype=torch.float32, device=dev)
     mb = w.mini_batch
+    if w.kind == "mlp":
+        run = [host[k].to(dev) for k in ("W1_0", "b1_0", "W2_0", "b2_0")]
+        start = [x.clone() for x in run]
 
-    def step(t, pos0, s):
-        ttt.ttt_linear_decode(t["Q"], t["K"], t["V"], t["eta"], W, b, W_mb, b_mb, gam, bet, pos0=pos0,
-                              mini_batch=mb, ln_eps=w.ln_eps, Z=Z, stream=s)
+        def step(t, pos0, s):
+            ttt.ttt_mlp_decode(t["Q"], t["K"], t["V"], t["eta"], *run, *start, gam, bet, pos0=pos0,
+                               mini_batch=mb, ln_eps=w.ln_eps, Z=Z, stream=s)
+    else:
+        W, b = host["W0"].to(dev), host["b0"].to(dev)
+        W_mb, b_mb = W.clone(), b.clone()
+
+        def step(t, pos0, s):
+            ttt.ttt_linear_decode(t["Q"], t["K"], t["V"], t["eta"], W, b, W_mb, b_mb, gam, bet, pos0=pos0,
+                                  mini_batch=mb, ln_eps=w.ln_eps, Z=Z, stream=s)
 
     # Device rate: one mini-batch cycle of single-token steps (positions 0..b-1)
     # captured in a CUDA graph, replayed; a decode loop runs this way.
@@ -397,6 +424,8 @@ def run_decode(args, world, rank, local):
     if rank == 0:
         hbm, _, peak_kind = load_peaks()
         ab = decode_state_bytes(w)
+        kname = ("ttt_mlp_generic_kernel" if w.kind == "mlp" else
+                 "ttt_linear_decode_kernel" if w.d == 64 else "ttt_linear_generic_kernel")
         achieved = ab / (kernel_ms * 1e-3) / 1e9
         line = {
             "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -405,16 +434,15 @@ def run_decode(args, world, rank, local):
             "data": "synthetic", "config": workload_config(w),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm,
-                         "traffic": recorded_traffic("ttt_linear_decode_kernel", w.name) if w.d == 64 else None,
+                         "traffic": recorded_traffic(kname, w.name),
                          "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms,
-                         "kernel": "ttt_linear_decode_kernel" if w.d == 64 else "ttt_linear_generic_kernel"},
+                         "algorithmic_bytes_per_launch": ab, "kernel_ms": kernel_ms, "kernel": kname},
             "cpu_baseline": cpu_base,
             "e2e": {"value": w.B * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": timed_steps,
             "clocks": clk.summary(),
-            "kernel_impl": "decode" if w.d == 64 else "generic",
+            "kernel_impl": "generic" if kname.endswith("generic_kernel") else "decode",
             "timing": "CUDA graph of one mini-batch cycle of steps, replayed; e2e: eager calls",
         }
         print(json.dumps(line), flush=True)
@@ -424,7 +452,7 @@ def run_ours(args, world, rank, local):
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
     w = WORKLOADS[args.workload]
-    if w.name == "decode_1p3b":
+    if w.name in DECODE_WORKLOADS:
         return run_decode(args, world, rank, local)
     dev = torch.device("cuda", local)
     host = make_inputs(w, args.seed + rank)
@@ -545,7 +573,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
-                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k == "decode_1p3b"])
+                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS])
     ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split"], default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,

@@ -188,6 +188,26 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
                                 float* W1_T, float* b1_T, float* W2_T, float* b2_T, ttt_impl impl,
                                 ttt_stream_t stream);
 
+/*
+ * TTT-MLP decode: the scan of ttt_mlp_forward continued by T >= 0 more tokens,
+ * the first at position pos0 of its mini-batch (0 <= pos0 < mini_batch, else
+ * TTT_ERR_SHAPE), as ttt_linear_decode for the linear model.
+ *   W1, b1, W2, b2          running state (shapes of ttt_mlp_forward's W1_0 ...),
+ *                           read, then overwritten with the state after the
+ *                           call's last token
+ *   W1_mb, b1_mb, W2_mb, b2_mb  state the current mini-batch started from: read
+ *                           when pos0 > 0, then overwritten with the start state
+ *                           of the mini-batch the next token falls in
+ * The eight state buffers, Z and the inputs must not overlap (TTT_ERR_ALIAS).
+ * Runs the generic fp32 family.
+ */
+ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
+                          ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
+                          const void* V, const float* eta, float* W1, float* b1, float* W2,
+                          float* b2, float* W1_mb, float* b1_mb, float* W2_mb, float* b2_mb,
+                          const float* ln_gamma, const float* ln_beta, float* Z,
+                          ttt_stream_t stream);
+
 /* Kernel family TTT_IMPL_AUTO would run for these TTT-MLP arguments
  * (TTT_IMPL_AUTO if no family covers them).  Pure host query.  Among the
  * tensor-core families it picks TTT_IMPL_TENSORCORE_SPLIT while the doubled

@@ -59,6 +59,8 @@ lib.ttt_linear_pick_impl.restype = _I
 lib.ttt_linear_pick_impl.argtypes = [_I] * 7
 lib.ttt_linear_decode.restype = _I
 lib.ttt_linear_decode.argtypes = [_I] * 8 + [_F] + [_P] * 11 + [_P]
+lib.ttt_mlp_decode.restype = _I
+lib.ttt_mlp_decode.argtypes = [_I] * 8 + [_F] + [_P] * 15 + [_P]
 
 
 def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
@@ -274,6 +276,36 @@ def ttt_linear_decode(Q, K, V, eta, W, b, W_mb, b_mb, ln_gamma=None, ln_beta=Non
         B, H, T, d, int(mini_batch), int(pos0), _dtype_code(Q), m, float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
         _ptr(eta), _ptr(W), _ptr(b), _ptr(W_mb), _ptr(b_mb), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z),
         _stream_handle(dev, stream))
+    _check(st)
+    return Z
+
+
+def ttt_mlp_decode(Q, K, V, eta, W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb, ln_gamma, ln_beta, *,
+                   pos0: int, mini_batch: int = 16, ln_eps: float = 1e-6, Z=None, stream=None) -> torch.Tensor:
+    """TTT-MLP decode (see include/ttt.h): the scan continued by T tokens from
+    position pos0 of a mini-batch.  The running state (W1, b1, W2, b2) and the
+    mini-batch start state (W1_mb, ...) are CUDA tensors updated in place.
+    Returns Z."""
+    B, H, T, d = Q.shape
+    state = (W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb)
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("eta", eta), ("ln_gamma", ln_gamma), ("ln_beta", ln_beta),
+                    *zip(("W1", "b1", "W2", "b2", "W1_mb", "b1_mb", "W2_mb", "b2_mb"), state)):
+        if t is None or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if K.shape != Q.shape or V.shape != Q.shape or K.dtype != Q.dtype or V.dtype != Q.dtype:
+        raise ValueError("Q, K, V must share shape and dtype")
+    hidden = W1.shape[-1]
+    shapes = ((B, H, d, hidden), (B, H, hidden), (B, H, hidden, d), (B, H, d)) * 2
+    if tuple(eta.shape) != (B, H, T) or any(tuple(t.shape) != sh for t, sh in zip(state, shapes)):
+        raise ValueError("eta must be [B,H,T]; W1 [B,H,d,hid], b1 [B,H,hid], W2 [B,H,hid,d], b2 [B,H,d]")
+    if any(t.dtype != torch.float32 for t in (eta, *state)):
+        raise TypeError("eta and the state must be float32")
+    dev = Q.device
+    if Z is None:
+        Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    st = lib.ttt_mlp_decode(
+        B, H, T, d, hidden, int(mini_batch), int(pos0), _dtype_code(Q), float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
+        _ptr(eta), *(_ptr(t) for t in state), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _stream_handle(dev, stream))
     _check(st)
     return Z
 

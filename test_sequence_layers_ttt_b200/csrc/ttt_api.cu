@@ -128,6 +128,28 @@ ttt_status validate_mlp(const MlpArgs& a) {
     return check_aliasing(outs, 5, ins, same_as, 10);
 }
 
+// TTT-MLP decode: the forward scan's checks with the running state in place,
+// plus the position and the mini-batch start state (read and written in place).
+ttt_status validate_mlp_decode(const MlpArgs& a) {
+    ttt_status st = validate_mlp(a);
+    if (st != TTT_OK) return st;
+    if (a.pos0 < 0 || a.pos0 >= a.mini_batch) return TTT_ERR_SHAPE;
+    const void* mb[] = {a.W1_mb, a.b1_mb, a.W2_mb, a.b2_mb};
+    for (const void* p : mb) {
+        if (!p) return TTT_ERR_NULL;
+        if (!aligned16(p)) return TTT_ERR_ALIGN;
+    }
+    const size_t es = a.dtype == TTT_BF16 ? 2 : 4;
+    const size_t bh = (size_t)a.B * a.H, ntok = bh * (size_t)a.T, d = a.d, hd = a.hidden;
+    Span ins[] = {{a.Q, ntok * d * es}, {a.K, ntok * d * es}, {a.V, ntok * d * es}, {a.eta, ntok * 4},
+                  {a.gamma, (size_t)a.H * d * 4}, {a.beta, (size_t)a.H * d * 4}};
+    Span outs[] = {{a.Z, ntok * d * 4},     {a.W1_T, bh * d * hd * 4},  {a.b1_T, bh * hd * 4},
+                   {a.W2_T, bh * hd * d * 4}, {a.b2_T, bh * d * 4},      {a.W1_mb, bh * d * hd * 4},
+                   {a.b1_mb, bh * hd * 4},   {a.W2_mb, bh * hd * d * 4}, {a.b2_mb, bh * d * 4}};
+    const int same_as[] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    return check_aliasing(outs, 9, ins, same_as, 6);
+}
+
 }  // namespace
 
 extern "C" {
@@ -220,6 +242,19 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
         default:
             return TTT_ERR_UNSUPPORTED;
     }
+}
+
+ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
+                          ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K, const void* V,
+                          const float* eta, float* W1, float* b1, float* W2, float* b2, float* W1_mb,
+                          float* b1_mb, float* W2_mb, float* b2_mb, const float* ln_gamma,
+                          const float* ln_beta, float* Z, ttt_stream_t stream) {
+    MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1, b1, W2, b2,
+              ln_gamma, ln_beta, Z, W1, b1, W2, b2, pos0, W1_mb, b1_mb, W2_mb, b2_mb};
+    ttt_status st = validate_mlp_decode(a);
+    if (st != TTT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return finish(ttt::launch_mlp_generic(a, s), s);
 }
 
 ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch, ttt_dtype qkv_dtype) {

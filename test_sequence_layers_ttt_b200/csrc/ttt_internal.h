@@ -29,6 +29,11 @@ struct MlpArgs {
     const void *Q, *K, *V;
     const float *eta, *W1_0, *b1_0, *W2_0, *b2_0, *gamma, *beta;
     float *Z, *W1_T, *b1_T, *W2_T, *b2_T;
+    // decode only (generic family): position of the first token in its
+    // mini-batch, and the mini-batch start state, read when pos0 > 0 and
+    // written in place
+    int pos0;
+    float *W1_mb, *b1_mb, *W2_mb, *b2_mb;
 };
 
 bool linear_generic_supports(const LinearArgs& a);

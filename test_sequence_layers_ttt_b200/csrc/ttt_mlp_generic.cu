@@ -18,6 +18,11 @@
 //           b2_c -= eta^T G2.
 // When b > 16 the start state lives in W1_T/b1_T/W2_T/b2_T (the caller's
 // final-state buffers) while the running state stays in shared memory.
+//
+// Decode (the scan continued by T tokens from position pos0 of a mini-batch):
+// the start state lives in the caller's W*_mb buffers (read when pos0 > 0),
+// the chunks are aligned to the stream's mini-batches, and W*_mb is left as
+// the start state of the mini-batch the next token falls in.
 #include "common.cuh"
 #include "ttt_internal.h"
 
@@ -51,19 +56,22 @@ ttt_mlp_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict__ 
                        const float* __restrict__ eta, const float* W1_0, const float* b1_0,
                        const float* W2_0, const float* b2_0, const float* __restrict__ gamma,
                        const float* __restrict__ beta, float* __restrict__ Z, float* W1_T,
-                       float* b1_T, float* W2_T, float* b2_T) {
+                       float* b1_T, float* W2_T, float* b2_T, int pos0, float* W1_mb, float* b1_mb,
+                       float* W2_mb, float* b2_mb) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     MlpSmem& s = *reinterpret_cast<MlpSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long bh = blockIdx.x;
     const int h = (int)(bh % H);
     const int C = mb < kChunk ? mb : kChunk;
-    const bool start_in_global = mb > kChunk;
+    const bool decode = W1_mb != nullptr;
+    const bool start_in_global = decode || mb > kChunk;
 
-    float* gW1 = W1_T + bh * D * HID;
-    float* gW2 = W2_T + bh * HID * D;
-    float* gb1 = b1_T + bh * HID;
-    float* gb2 = b2_T + bh * D;
+    // global start-state buffers: the caller's W*_mb (decode) or W*_T (b > 16)
+    float* gW1 = (decode ? W1_mb : W1_T) + bh * D * HID;
+    float* gW2 = (decode ? W2_mb : W2_T) + bh * HID * D;
+    float* gb1 = (decode ? b1_mb : b1_T) + bh * HID;
+    float* gb2 = (decode ? b2_mb : b2_T) + bh * D;
     for (int i = tid; i < D * HID; i += kThreads) s.W1c[i] = W1_0[bh * D * HID + i];
     for (int i = tid; i < HID * D; i += kThreads) s.W2c[(i / D) * LDW2 + i % D] = W2_0[bh * HID * D + i];
     for (int k = tid; k < HID; k += kThreads) s.b1c[k] = b1_0[bh * HID + k];
@@ -80,10 +88,11 @@ ttt_mlp_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict__ 
     const float* b2s = start_in_global ? gb2 : s.b2c;
 
     const long tok0 = bh * (long)T;
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int n = min(C, T - t0);
+    for (int t0 = 0, n = 0; t0 < T; t0 += n) {
+        const int ph = (pos0 + t0) % mb;  // position of the chunk's first token in its mini-batch
+        n = min(min(C, T - t0), mb - ph);
         __syncthreads();
-        if (start_in_global && t0 % mb == 0) {
+        if (start_in_global && ph == 0) {
             for (int i = tid; i < D * HID; i += kThreads) gW1[i] = s.W1c[i];
             for (int i = tid; i < HID * D; i += kThreads) gW2[i] = s.W2c[(i / D) * LDW2 + i % D];
             for (int k = tid; k < HID; k += kThreads) gb1[k] = s.b1c[k];
@@ -278,10 +287,20 @@ ttt_mlp_generic_kernel(int H, int T, int mb, float eps, const Tin* __restrict__ 
         }
     }
     __syncthreads();
-    for (int i = tid; i < D * HID; i += kThreads) gW1[i] = s.W1c[i];
-    for (int i = tid; i < HID * D; i += kThreads) gW2[i] = s.W2c[(i / D) * LDW2 + i % D];
-    for (int k = tid; k < HID; k += kThreads) gb1[k] = s.b1c[k];
-    for (int j = tid; j < D; j += kThreads) gb2[j] = s.b2c[j];
+    float* oW1 = W1_T + bh * D * HID;
+    float* oW2 = W2_T + bh * HID * D;
+    float* ob1 = b1_T + bh * HID;
+    float* ob2 = b2_T + bh * D;
+    for (int i = tid; i < D * HID; i += kThreads) oW1[i] = s.W1c[i];
+    for (int i = tid; i < HID * D; i += kThreads) oW2[i] = s.W2c[(i / D) * LDW2 + i % D];
+    for (int k = tid; k < HID; k += kThreads) ob1[k] = s.b1c[k];
+    for (int j = tid; j < D; j += kThreads) ob2[j] = s.b2c[j];
+    if (decode && (pos0 + T) % mb == 0) {  // the next token starts a mini-batch from the final state
+        for (int i = tid; i < D * HID; i += kThreads) gW1[i] = s.W1c[i];
+        for (int i = tid; i < HID * D; i += kThreads) gW2[i] = s.W2c[(i / D) * LDW2 + i % D];
+        for (int k = tid; k < HID; k += kThreads) gb1[k] = s.b1c[k];
+        for (int j = tid; j < D; j += kThreads) gb2[j] = s.b2c[j];
+    }
 }
 
 template <typename Tin>
@@ -293,7 +312,7 @@ cudaError_t launch_t(const MlpArgs& a, cudaStream_t stream) {
     kern<<<a.B * a.H, kThreads, smem, stream>>>(
         a.H, a.T, a.mini_batch, a.ln_eps, static_cast<const Tin*>(a.Q), static_cast<const Tin*>(a.K),
         static_cast<const Tin*>(a.V), a.eta, a.W1_0, a.b1_0, a.W2_0, a.b2_0, a.gamma, a.beta, a.Z,
-        a.W1_T, a.b1_T, a.W2_T, a.b2_T);
+        a.W1_T, a.b1_T, a.W2_T, a.b2_T, a.pos0, a.W1_mb, a.b1_mb, a.W2_mb, a.b2_mb);
     return cudaPeekAtLastError();
 }
 

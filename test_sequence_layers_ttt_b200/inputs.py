@@ -64,6 +64,8 @@ WORKLOADS: Dict[str, Workload] = {
     # Decode on the 1.3B-class layer: the stream of B=2 sequences x H=32 heads
     # continued one token per step; T is the number of tokens generated.
     "decode_1p3b": Workload("decode_1p3b", "linear", 2, 32, 256, 64, 16, "bf16", init="lm"),
+    # Decode on the TTT-MLP layer: B=4 x H=12 streams, one token per step.
+    "decode_mlp_8k": Workload("decode_mlp_8k", "mlp", 4, 12, 256, 64, 16, "bf16", hidden=256, init="mlp"),
     # TTT-MLP layer: B=4, H=12, d=64, 64 -> 256 -> 64, T=8192, b=16.
     "mlp_8k": Workload("mlp_8k", "mlp", 4, 12, 8192, 64, 16, "bf16", hidden=256, init="mlp"),
 }

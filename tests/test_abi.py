@@ -171,6 +171,34 @@ def test_decode_overlapping_buffers(dst, src, off):
     assert decode_call(ptrs=p) == ALIAS
 
 
+# MLP decode: Q K V eta W1 b1 W2 b2 W1_mb b1_mb W2_mb b2_mb gamma beta Z
+def mlp_decode_call(B=1, H=2, T=64, mb=16, pos0=0, ptrs=None):
+    p = [fake(i) for i in range(15)] if ptrs is None else ptrs
+    return b.lib.ttt_mlp_decode(B, H, T, 64, 256, mb, pos0, 0, 1e-6, *p, None)
+
+
+@pytest.mark.parametrize("pos0", [-1, 16])
+def test_mlp_decode_position_outside_the_mini_batch(pos0):
+    assert mlp_decode_call(pos0=pos0) == SHAPE
+
+
+@pytest.mark.parametrize("idx", [4, 8, 9, 10, 11])
+def test_mlp_decode_null_state(idx):
+    assert mlp_decode_call(ptrs=with_ptr(idx, None, 15)) == NULL
+
+
+@pytest.mark.parametrize("idx", [8, 9, 10, 11])
+def test_mlp_decode_misaligned_start_state(idx):
+    assert mlp_decode_call(ptrs=with_ptr(idx, fake(idx) + 4, 15)) == ALIGN
+
+
+@pytest.mark.parametrize("dst,src,off", [(8, 4, 256), (11, 14, 0), (10, 0, 64), (9, 5, 0)])
+def test_mlp_decode_overlapping_buffers(dst, src, off):
+    p = [fake(k) for k in range(15)]
+    p[dst] = p[src] + off
+    assert mlp_decode_call(ptrs=p) == ALIAS
+
+
 def test_linear_has_no_split_family():
     # the split family is TTT-MLP only; unknown families are refused before any launch
     assert linear_call(impl=3) == UNSUP

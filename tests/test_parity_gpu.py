@@ -431,6 +431,81 @@ def compare_mlp(ttt, w, inp, mini_batch=None, pairs=None, impl="auto"):
         assert_close(o, r, f, name, denom=max(scale, 1e-3 * rms(ref[1])))
 
 
+STATE_MLP = ("W1_0", "b1_0", "W2_0", "b2_0")
+
+
+def gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb):
+    g = to_cuda(inp)
+    run = [g[k].clone() for k in STATE_MLP]
+    start = [torch.zeros_like(x) for x in run]
+    T = g["Q"].shape[2]
+    bounds = [0, *cuts, T]
+    Zs = []
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = lambda x: x[:, :, a:c].contiguous()
+        Zs.append(ttt.ttt_mlp_decode(sl(g["Q"]), sl(g["K"]), sl(g["V"]), sl(g["eta"]), *run, *start, g["gamma"],
+                                     g["beta"], pos0=a % mb, mini_batch=mb, ln_eps=w.ln_eps))
+    torch.cuda.synchronize()
+    return [x.cpu().numpy() for x in (torch.cat(Zs, dim=2), *run, *start)]
+
+
+def oracle_mlp_decode_pieces(w, inp, cuts, mb):
+    T = inp["Q"].shape[2]
+    run, start = [inp[k] for k in STATE_MLP], [None] * 4
+    bounds = [0, *cuts, T]
+    Zs = []
+    for a, c in zip(bounds[:-1], bounds[1:]):
+        sl = lambda x: x[:, :, a:c]
+        out = oracle.ttt_mlp_decode(sl(inp["Q"]), sl(inp["K"]), sl(inp["V"]), sl(inp["eta"]), *run, *start,
+                                    inp["gamma"], inp["beta"], mb, a % mb, w.ln_eps)
+        Zs.append(out[0])
+        run, start = list(out[1:5]), list(out[5:9])
+    return [np.concatenate(Zs, axis=2), *run, *start]
+
+
+@pytest.mark.parametrize("shape,mb,cuts", [
+    (dict(B=1, H=2, T=80), 16, [5, 6, 21, 40, 63]),
+    (dict(B=1, H=2, T=72), 32, [1, 33, 50]),
+    (dict(B=1, H=2, T=40), 8, [3, 4, 19]),
+    (dict(B=1, H=2, T=48, dtype="f32"), 16, [7, 30]),
+])
+def test_mlp_decode_pieces_vs_oracle(ttt, shape, mb, cuts):
+    """TTT-MLP decode calls cut anywhere against the oracle's decode over the same
+    pieces: outputs, running state and mini-batch start state."""
+    w = WORKLOADS["mlp_8k"].with_shape(**shape)
+    inp = make_inputs(w, 3)
+    out = gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb)
+    ref = oracle_mlp_decode_pieces(w, inp, cuts, mb)
+    f = TOL[w.dtype]
+    assert_close(out[0], ref[0], f, "Z")
+    names = ("W1", "b1", "W2", "b2", "W1_mb", "b1_mb", "W2_mb", "b2_mb")
+    for name, o, r in zip(names, out[1:], ref[1:]):
+        scale = rms(r) if np.any(r) else 1.0
+        assert_close(o, r, f, name, denom=max(scale, 1e-3 * rms(ref[1])))
+
+
+def test_mlp_decode_token_by_token_equals_forward_oracle(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=24)
+    inp = make_inputs(w, 4)
+    out = gpu_mlp_decode_pieces(ttt, w, inp, list(range(1, 24)), 16)
+    ref = oracle_mlp(w, inp)
+    assert_close(out[0], ref[0], TOL[w.dtype], "Z")
+
+
+def test_mlp_decode_one_call_is_the_generic_forward(ttt):
+    """From a mini-batch boundary, one decode call runs the generic forward scan
+    operation for operation (the start state read from the caller's buffer
+    instead of shared memory)."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=64)
+    inp = make_inputs(w, 5)
+    dec = gpu_mlp_decode_pieces(ttt, w, inp, [], 16)
+    fwd = gpu_mlp(ttt, w, inp, impl="generic")
+    for a, b in zip(dec[:5], fwd):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(dec[5:], fwd[1:]):  # T = 64 ends on a boundary: the next mini-batch starts from W_T
+        np.testing.assert_array_equal(a, b)
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_mlp_reduced(ttt, seed):
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=200)
