@@ -351,11 +351,11 @@ def run_decode(args, world, rank, local):
     Z = torch.empty((w.B, w.H, 1, w.d), dtype=torch.float32, device=dev)
     mb = w.mini_batch
     if w.kind == "mlp":
-        run = [host[k].to(dev) for k in ("W1_0", "b1_0", "W2_0", "b2_0")]
-        start = [x.clone() for x in run]
+        mlp_run = [host[k].to(dev) for k in ("W1_0", "b1_0", "W2_0", "b2_0")]
+        mlp_start = [x.clone() for x in mlp_run]
 
         def step(t, pos0, s):
-            ttt.ttt_mlp_decode(t["Q"], t["K"], t["V"], t["eta"], *run, *start, gam, bet, pos0=pos0,
+            ttt.ttt_mlp_decode(t["Q"], t["K"], t["V"], t["eta"], *mlp_run, *mlp_start, gam, bet, pos0=pos0,
                                mini_batch=mb, ln_eps=w.ln_eps, Z=Z, stream=s)
     else:
         W, b = host["W0"].to(dev), host["b0"].to(dev)
