@@ -90,6 +90,7 @@ KERNEL_SOURCES = {
     "ttt_mlp_split_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_generic_kernel": ("ttt_mlp_generic.cu", "common.cuh", "ttt_internal.h"),
     "ttt_linear_decode_kernel": ("ttt_linear_decode.cu", "common.cuh", "ttt_internal.h"),
+    "ttt_mlp_decode_kernel": ("ttt_mlp_decode.cu", "common.cuh", "ttt_internal.h"),
 }
 
 
@@ -424,7 +425,7 @@ def run_decode(args, world, rank, local):
     if rank == 0:
         hbm, _, peak_kind = load_peaks()
         ab = decode_state_bytes(w)
-        kname = ("ttt_mlp_generic_kernel" if w.kind == "mlp" else
+        kname = ("ttt_mlp_decode_kernel" if w.kind == "mlp" else
                  "ttt_linear_decode_kernel" if w.d == 64 else "ttt_linear_generic_kernel")
         achieved = ab / (kernel_ms * 1e-3) / 1e9
         line = {

@@ -199,7 +199,8 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
  *                           when pos0 > 0, then overwritten with the start state
  *                           of the mini-batch the next token falls in
  * The eight state buffers, Z and the inputs must not overlap (TTT_ERR_ALIAS).
- * Runs the generic fp32 family.
+ * Runs a decode kernel that keeps the running state in registers for the
+ * whole call (token-serial, fp32).
  */
 ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
                           ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
@@ -207,6 +208,16 @@ ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch
                           float* b2, float* W1_mb, float* b1_mb, float* W2_mb, float* b2_mb,
                           const float* ln_gamma, const float* ln_beta, float* Z,
                           ttt_stream_t stream);
+
+/* As ttt_mlp_decode with an explicit family: TTT_IMPL_AUTO (the decode kernel)
+ * or TTT_IMPL_GENERIC (the generic fp32 scan run from inside a mini-batch);
+ * TTT_ERR_UNSUPPORTED for any other. */
+ttt_status ttt_mlp_decode_impl(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
+                               ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K,
+                               const void* V, const float* eta, float* W1, float* b1, float* W2,
+                               float* b2, float* W1_mb, float* b1_mb, float* W2_mb, float* b2_mb,
+                               const float* ln_gamma, const float* ln_beta, float* Z, ttt_impl impl,
+                               ttt_stream_t stream);
 
 /* Kernel family TTT_IMPL_AUTO would run for these TTT-MLP arguments
  * (TTT_IMPL_AUTO if no family covers them).  Pure host query.  Among the

@@ -61,6 +61,8 @@ lib.ttt_linear_decode.restype = _I
 lib.ttt_linear_decode.argtypes = [_I] * 8 + [_F] + [_P] * 11 + [_P]
 lib.ttt_mlp_decode.restype = _I
 lib.ttt_mlp_decode.argtypes = [_I] * 8 + [_F] + [_P] * 15 + [_P]
+lib.ttt_mlp_decode_impl.restype = _I
+lib.ttt_mlp_decode_impl.argtypes = [_I] * 8 + [_F] + [_P] * 15 + [_I, _P]
 
 
 def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
@@ -281,7 +283,8 @@ def ttt_linear_decode(Q, K, V, eta, W, b, W_mb, b_mb, ln_gamma=None, ln_beta=Non
 
 
 def ttt_mlp_decode(Q, K, V, eta, W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb, ln_gamma, ln_beta, *,
-                   pos0: int, mini_batch: int = 16, ln_eps: float = 1e-6, Z=None, stream=None) -> torch.Tensor:
+                   pos0: int, mini_batch: int = 16, ln_eps: float = 1e-6, impl: str = "auto", Z=None,
+                   stream=None) -> torch.Tensor:
     """TTT-MLP decode (see include/ttt.h): the scan continued by T tokens from
     position pos0 of a mini-batch.  The running state (W1, b1, W2, b2) and the
     mini-batch start state (W1_mb, ...) are CUDA tensors updated in place.
@@ -303,9 +306,10 @@ def ttt_mlp_decode(Q, K, V, eta, W1, b1, W2, b2, W1_mb, b1_mb, W2_mb, b2_mb, ln_
     dev = Q.device
     if Z is None:
         Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
-    st = lib.ttt_mlp_decode(
+    st = lib.ttt_mlp_decode_impl(
         B, H, T, d, hidden, int(mini_batch), int(pos0), _dtype_code(Q), float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
-        _ptr(eta), *(_ptr(t) for t in state), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _stream_handle(dev, stream))
+        _ptr(eta), *(_ptr(t) for t in state), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), IMPLS[impl],
+        _stream_handle(dev, stream))
     _check(st)
     return Z
 

@@ -8,6 +8,13 @@
 
 #include "ttt_internal.h"
 
+namespace ttt {
+// TTT-MLP decode with the running state in registers (d = 64, hidden = 256),
+// in place on W*_T / b*_T and W*_mb / b*_mb (ttt_mlp_decode.cu).
+bool mlp_decode_supports(const MlpArgs& a);
+cudaError_t launch_mlp_decode(const MlpArgs& a, cudaStream_t stream);
+}  // namespace ttt
+
 namespace {
 
 using ttt::LinearArgs;
@@ -244,17 +251,34 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
     }
 }
 
-ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
-                          ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K, const void* V,
-                          const float* eta, float* W1, float* b1, float* W2, float* b2, float* W1_mb,
-                          float* b1_mb, float* W2_mb, float* b2_mb, const float* ln_gamma,
-                          const float* ln_beta, float* Z, ttt_stream_t stream) {
+ttt_status ttt_mlp_decode_impl(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
+                               ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K, const void* V,
+                               const float* eta, float* W1, float* b1, float* W2, float* b2, float* W1_mb,
+                               float* b1_mb, float* W2_mb, float* b2_mb, const float* ln_gamma,
+                               const float* ln_beta, float* Z, ttt_impl impl, ttt_stream_t stream) {
     MlpArgs a{B, H, T, d, hidden, mini_batch, qkv_dtype, ln_eps, Q, K, V, eta, W1, b1, W2, b2,
               ln_gamma, ln_beta, Z, W1, b1, W2, b2, pos0, W1_mb, b1_mb, W2_mb, b2_mb};
     ttt_status st = validate_mlp_decode(a);
     if (st != TTT_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return finish(ttt::launch_mlp_generic(a, s), s);
+    switch (impl) {
+        case TTT_IMPL_AUTO:
+            if (ttt::mlp_decode_supports(a)) return finish(ttt::launch_mlp_decode(a, s), s);
+            return finish(ttt::launch_mlp_generic(a, s), s);
+        case TTT_IMPL_GENERIC:
+            return finish(ttt::launch_mlp_generic(a, s), s);
+        default:
+            return TTT_ERR_UNSUPPORTED;
+    }
+}
+
+ttt_status ttt_mlp_decode(int B, int H, int T, int d, int hidden, int mini_batch, int pos0,
+                          ttt_dtype qkv_dtype, float ln_eps, const void* Q, const void* K, const void* V,
+                          const float* eta, float* W1, float* b1, float* W2, float* b2, float* W1_mb,
+                          float* b1_mb, float* W2_mb, float* b2_mb, const float* ln_gamma,
+                          const float* ln_beta, float* Z, ttt_stream_t stream) {
+    return ttt_mlp_decode_impl(B, H, T, d, hidden, mini_batch, pos0, qkv_dtype, ln_eps, Q, K, V, eta, W1, b1,
+                               W2, b2, W1_mb, b1_mb, W2_mb, b2_mb, ln_gamma, ln_beta, Z, TTT_IMPL_AUTO, stream);
 }
 
 ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch, ttt_dtype qkv_dtype) {

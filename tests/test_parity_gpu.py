@@ -434,7 +434,7 @@ def compare_mlp(ttt, w, inp, mini_batch=None, pairs=None, impl="auto"):
 STATE_MLP = ("W1_0", "b1_0", "W2_0", "b2_0")
 
 
-def gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb):
+def gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb, impl="auto"):
     g = to_cuda(inp)
     run = [g[k].clone() for k in STATE_MLP]
     start = [torch.zeros_like(x) for x in run]
@@ -444,7 +444,7 @@ def gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb):
     for a, c in zip(bounds[:-1], bounds[1:]):
         sl = lambda x: x[:, :, a:c].contiguous()
         Zs.append(ttt.ttt_mlp_decode(sl(g["Q"]), sl(g["K"]), sl(g["V"]), sl(g["eta"]), *run, *start, g["gamma"],
-                                     g["beta"], pos0=a % mb, mini_batch=mb, ln_eps=w.ln_eps))
+                                     g["beta"], pos0=a % mb, mini_batch=mb, ln_eps=w.ln_eps, impl=impl))
     torch.cuda.synchronize()
     return [x.cpu().numpy() for x in (torch.cat(Zs, dim=2), *run, *start)]
 
@@ -463,18 +463,23 @@ def oracle_mlp_decode_pieces(w, inp, cuts, mb):
     return [np.concatenate(Zs, axis=2), *run, *start]
 
 
-@pytest.mark.parametrize("shape,mb,cuts", [
-    (dict(B=1, H=2, T=80), 16, [5, 6, 21, 40, 63]),
-    (dict(B=1, H=2, T=72), 32, [1, 33, 50]),
-    (dict(B=1, H=2, T=40), 8, [3, 4, 19]),
-    (dict(B=1, H=2, T=48, dtype="f32"), 16, [7, 30]),
+@pytest.mark.parametrize("shape,mb,cuts,impl", [
+    (dict(B=1, H=2, T=80), 16, [5, 6, 21, 40, 63], "auto"),
+    (dict(B=1, H=2, T=72), 32, [1, 33, 50], "auto"),
+    (dict(B=1, H=2, T=40), 8, [3, 4, 19], "auto"),
+    (dict(B=1, H=2, T=24), 1, [5, 9], "auto"),
+    (dict(B=1, H=2, T=48, dtype="f32"), 16, [7, 30], "auto"),
+    (dict(B=2, H=3, T=40), 16, [5, 21], "auto"),
+    (dict(B=1, H=2, T=80), 16, [5, 6, 21, 40, 63], "generic"),
+    (dict(B=1, H=2, T=72), 32, [1, 33, 50], "generic"),
 ])
-def test_mlp_decode_pieces_vs_oracle(ttt, shape, mb, cuts):
+def test_mlp_decode_pieces_vs_oracle(ttt, shape, mb, cuts, impl):
     """TTT-MLP decode calls cut anywhere against the oracle's decode over the same
-    pieces: outputs, running state and mini-batch start state."""
+    pieces: outputs, running state and mini-batch start state (the decode kernel,
+    and the generic scan run from inside a mini-batch)."""
     w = WORKLOADS["mlp_8k"].with_shape(**shape)
     inp = make_inputs(w, 3)
-    out = gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb)
+    out = gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb, impl)
     ref = oracle_mlp_decode_pieces(w, inp, cuts, mb)
     f = TOL[w.dtype]
     assert_close(out[0], ref[0], f, "Z")
@@ -492,13 +497,37 @@ def test_mlp_decode_token_by_token_equals_forward_oracle(ttt):
     assert_close(out[0], ref[0], TOL[w.dtype], "Z")
 
 
+def test_mlp_decode_register_kernel_matches_generic_forward(ttt):
+    """The decode kernel (running state in registers, token-serial) against the
+    generic forward scan: the same fp32 arithmetic in another order."""
+    w = WORKLOADS["mlp_8k"].with_shape(B=2, H=2, T=64)
+    inp = make_inputs(w, 6)
+    dec = gpu_mlp_decode_pieces(ttt, w, inp, [], 16)
+    fwd = gpu_mlp(ttt, w, inp, impl="generic")
+    for name, a, b in zip(("Z", "W1", "b1", "W2", "b2"), dec[:5], fwd):
+        assert_close(a, b.astype(np.float64), 1e-4, name, denom=max(rms(b), 1e-3))
+
+
+def test_mlp_decode_empty_call_keeps_state(ttt):
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=0)
+    g = to_cuda(make_inputs(w, 2))
+    run = [g[k].clone() for k in STATE_MLP]
+    start = [x + 0.5 for x in run]
+    start0 = [x.clone() for x in start]
+    Z = ttt.ttt_mlp_decode(g["Q"], g["K"], g["V"], g["eta"], *run, *start, g["gamma"], g["beta"], pos0=5)
+    torch.cuda.synchronize()
+    assert Z.shape == (1, 2, 0, 64)
+    assert all(torch.equal(a, g[k]) for a, k in zip(run, STATE_MLP))
+    assert all(torch.equal(a, b) for a, b in zip(start, start0))
+
+
 def test_mlp_decode_one_call_is_the_generic_forward(ttt):
-    """From a mini-batch boundary, one decode call runs the generic forward scan
-    operation for operation (the start state read from the caller's buffer
-    instead of shared memory)."""
+    """From a mini-batch boundary, one generic decode call runs the generic
+    forward scan operation for operation (the start state read from the
+    caller's buffer instead of shared memory)."""
     w = WORKLOADS["mlp_8k"].with_shape(B=1, H=2, T=64)
     inp = make_inputs(w, 5)
-    dec = gpu_mlp_decode_pieces(ttt, w, inp, [], 16)
+    dec = gpu_mlp_decode_pieces(ttt, w, inp, [], 16, impl="generic")
     fwd = gpu_mlp(ttt, w, inp, impl="generic")
     for a, b in zip(dec[:5], fwd):
         np.testing.assert_array_equal(a, b)
