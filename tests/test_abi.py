@@ -199,6 +199,14 @@ def test_mlp_decode_overlapping_buffers(dst, src, off):
     assert mlp_decode_call(ptrs=p) == ALIAS
 
 
+@pytest.mark.parametrize("impl", [2, 3, 9])
+def test_mlp_decode_families(impl):
+    # decode has the decode kernel (auto) and the generic scan; other families are
+    # refused after validation, before any launch
+    p = [fake(i) for i in range(15)]
+    assert b.lib.ttt_mlp_decode_impl(1, 2, 64, 64, 256, 16, 0, 0, 1e-6, *p, impl, None) == UNSUP
+
+
 def test_linear_has_no_split_family():
     # the split family is TTT-MLP only; unknown families are refused before any launch
     assert linear_call(impl=3) == UNSUP
