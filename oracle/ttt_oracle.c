@@ -13,7 +13,9 @@
  *
  * Parity pins (tests/test_oracle.py): Theorem 1 closed form, central finite
  * differences and autograd for every gradient, b = 1 against online GD,
- * eta = 0, state continuation, LayerNorm and GELU against library routines.
+ * eta = 0, state continuation, LayerNorm and GELU against library routines;
+ * decode (linear and MLP) in pieces against the mini-batch rule written out
+ * with autograd, and single-token plain decode against Theorem 1.
  */
 #include <math.h>
 #include <stdlib.h>
