@@ -1,4 +1,5 @@
-"""Float64 oracle of the TTT-Linear layer's backward (outer-loop gradients).
+"""Float64 oracle of the TTT layer's backward (outer-loop gradients), for
+TTT-Linear and (below) TTT-MLP.
 
 TEST INFRASTRUCTURE.  Only ``tests/`` may import this module; the CUDA library
 never calls it.
@@ -22,7 +23,8 @@ start state, running-state update, output with the running state), with the
 inner gradient computed in closed form (LayerNorm backward written out), and
 torch autograd applied to the whole scan as a library primitive.  Autograd
 then supplies the second-order terms (the update depends on W_s through the
-LayerNorm backward).
+LayerNorm backward).  For TTT-MLP the inner gradient itself is taken by
+autograd (with its graph kept), over the same loop.
 """
 from __future__ import annotations
 
@@ -131,3 +133,63 @@ def linear_forward(Q, K, V, eta, W0, b0, gamma, beta, mini_batch: int, mode: int
         Z, W_T, b_T = linear_scan(Qt, Kt, Vt, et, W0t, b0t, None if plain else _t(gamma),
                                   None if plain else _t(beta), mini_batch, mode, ln_eps)
         return Z.numpy(), W_T.numpy(), None if plain else b_T.numpy()
+
+
+# ---------------------------------------------------------------- TTT-MLP
+def _gelu(x):
+    # tanh form, as in the forward oracle
+    c = 0.7978845608028654
+    return 0.5 * x * (1.0 + torch.tanh(c * (x + 0.044715 * x ** 3)))
+
+
+def _ln_res(x, y, gamma, beta, eps):
+    mu = y.mean(-1, keepdim=True)
+    var = ((y - mu) ** 2).mean(-1, keepdim=True)
+    return x + gamma * (y - mu) / torch.sqrt(var + eps) + beta
+
+
+def mlp_scan(Q, K, V, eta, W1, b1, W2, b2, gamma, beta, mini_batch: int, eps: float):
+    """The TTT-MLP primal scan in float64 torch (differentiable; the inner
+    gradient by autograd with create_graph, so the outer gradient sees its
+    dependence on the state).  Shapes as the forward oracle's.  Returns
+    (Z, W1_T, b1_T, W2_T, b2_T)."""
+    B, H, T, d = Q.shape
+    g, be = gamma[None], beta[None]
+
+    def f(x, W1_, b1_, W2_, b2_):
+        a = _gelu(torch.einsum("bhi,bhij->bhj", x, W1_) + b1_)
+        return _ln_res(x, torch.einsum("bhi,bhij->bhj", a, W2_) + b2_, g, be, eps)
+
+    S = [W1, b1, W2, b2]
+    Zs = []
+    for m in range(0, T, mini_batch):
+        C = list(S)
+        for t in range(m, min(m + mini_batch, T)):
+            k, v, q = K[:, :, t], V[:, :, t], Q[:, :, t]
+            loss = ((f(k, *S) - v) ** 2).sum()
+            grads = torch.autograd.grad(loss, S, create_graph=True)
+            e = eta[:, :, t]
+            C = [c - (e[..., None, None] if c.dim() == 4 else e[..., None]) * gr for c, gr in zip(C, grads)]
+            Zs.append(f(q, *C))
+        S = C
+    return (torch.stack(Zs, dim=2), *S)
+
+
+def ttt_mlp_backward(Q, K, V, eta, W1, b1, W2, b2, gamma, beta, dZ, mini_batch: int,
+                     ln_eps: float = 1e-6, d_state=None):
+    """Gradients of sum(Z dZ) (+ sum over the final state times d_state, a
+    tuple (dW1_T, db1_T, dW2_T, db2_T)) with respect to (Q, K, V, eta, W1, b1,
+    W2, b2, gamma, beta)."""
+    ins = [_t(x, True) for x in (Q, K, V, eta, W1, b1, W2, b2, gamma, beta)]
+    out = mlp_scan(*ins, mini_batch, ln_eps)
+    L = (out[0] * _t(dZ)).sum()
+    if d_state is not None:
+        for s_, ds_ in zip(out[1:], d_state):
+            L = L + (s_ * _t(ds_)).sum()
+    return tuple(gr.numpy() for gr in torch.autograd.grad(L, ins))
+
+
+def mlp_forward(Q, K, V, eta, W1, b1, W2, b2, gamma, beta, mini_batch: int, ln_eps: float = 1e-6):
+    """The torch primal's outputs (for checking it against the C oracle)."""
+    ins = [_t(x, True) for x in (Q, K, V, eta, W1, b1, W2, b2, gamma, beta)]
+    return tuple(o.detach().numpy() for o in mlp_scan(*ins, mini_batch, ln_eps))

@@ -1,10 +1,10 @@
 """Pins of the float64 backward oracle (oracle/backward.py), CPU only.
 
-The backward oracle differentiates a torch restatement of the TTT-Linear
-scan.  These tests tie it to things other than itself:
-- its primal equals the C oracle's scan;
-- every gradient equals central finite differences of the C oracle;
-- in Theorem 1's setting (plain f, one mini-batch, W0 = 0; Key takeaways
+The backward oracle differentiates torch restatements of the TTT-Linear and
+TTT-MLP scans.  These tests tie it to things other than itself:
+- its primal equals the C oracle's scan (both models);
+- every gradient equals central finite differences of the C oracle (both);
+- for TTT-Linear, in Theorem 1's setting (plain f, one mini-batch, W0 = 0; Key takeaways
   bullet 3 of the literature record) the gradients have a closed form, that
   of causal linear attention with per-token weights 2 eta_s.
 """
@@ -110,3 +110,55 @@ def test_theorem1_gradients_closed_form():
         S += e[t] * np.outer(k[t], k[t])
         dW0 += (np.eye(d) - 2 * S) @ np.outer(q[t], dz[t])
     np.testing.assert_allclose(g[4][0, 0], dW0, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- TTT-MLP
+
+def mlp_case(seed, T=10, d=4, hid=6):
+    r = np.random.default_rng(seed)
+    Q, K, V = (r.normal(0, 1 / np.sqrt(d), (1, 1, T, d)) for _ in range(3))
+    eta = 1 / (1 + np.exp(-r.normal(0, 1, (1, 1, T)))) / d * 4
+    W1 = r.normal(0, 1 / np.sqrt(d), (1, 1, d, hid))
+    b1 = r.normal(0, 0.1, (1, 1, hid))
+    W2 = r.normal(0, 1 / np.sqrt(hid), (1, 1, hid, d))
+    b2 = r.normal(0, 0.1, (1, 1, d))
+    gamma = 1 + r.normal(0, 0.2, (1, d))
+    beta = r.normal(0, 0.2, (1, d))
+    dZ = r.normal(0, 1, (1, 1, T, d))
+    dS = (r.normal(0, 1, (1, 1, d, hid)), r.normal(0, 1, (1, 1, hid)), r.normal(0, 1, (1, 1, hid, d)),
+          r.normal(0, 1, (1, 1, d)))
+    return [Q, K, V, eta, W1, b1, W2, b2, gamma, beta], dZ, dS
+
+
+@pytest.mark.parametrize("mb,T", [(4, 10), (1, 5), (8, 8)])
+def test_mlp_torch_primal_equals_c_oracle(mb, T):
+    ins, _, _ = mlp_case(3, T=T)
+    got = ob.mlp_forward(*ins, mb)
+    ref = oracle.ttt_mlp(*ins, mb)
+    for g, r in zip(got, ref):
+        assert rel(g, r) < 1e-12
+
+
+def test_mlp_gradients_equal_finite_differences_of_the_c_oracle():
+    ins, dZ, dS = mlp_case(4)
+    mb = 4
+    grads = ob.ttt_mlp_backward(*ins, dZ, mb, d_state=dS)
+
+    def loss(xs):
+        out = oracle.ttt_mlp(*xs, mb)
+        return float((out[0] * dZ).sum() + sum((o * w).sum() for o, w in zip(out[1:], dS)))
+
+    names = ["Q", "K", "V", "eta", "W1", "b1", "W2", "b2", "gamma", "beta"]
+    h = 1e-6
+    for i, (name, x) in enumerate(zip(names, ins)):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            j = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[j] += h
+            xm[j] -= h
+            ip, im = list(ins), list(ins)
+            ip[i], im[i] = xp, xm
+            fd[j] = (loss(ip) - loss(im)) / (2 * h)
+        assert rel(grads[i], fd) < 1e-6, f"d{name}: {rel(grads[i], fd):.2e}"
