@@ -1,5 +1,6 @@
-"""The TTT-Linear layer backward as a backward kernel would run it, checked
-against the pinned float64 backward oracle (oracle/backward.py).  CPU only.
+"""The TTT layer backward (TTT-Linear, then TTT-MLP) as a backward kernel
+would run it, checked against the pinned float64 backward oracle
+(oracle/backward.py).  CPU only.
 
 A restatement of the algorithm, not a second oracle.  Forward: chunk by chunk
 (a chunk is one mini-batch of b <= 16 tokens) in the dual form, keeping each
@@ -148,3 +149,178 @@ def test_chunked_backward_equals_the_oracle(T, chunk):
     for name, g, r in zip(names, got, ref):
         r = r[0, 0] if name not in ("dgamma", "dbeta") else r[0]
         assert rel(g, r) < 1e-10, f"{name}: {rel(g, r):.2e}"
+
+
+# ---------------------------------------------------------------- TTT-MLP
+
+_C = 0.7978845608028654  # sqrt(2 / pi)
+
+
+def _gelu(x):
+    return 0.5 * x * (1.0 + np.tanh(_C * (x + 0.044715 * x ** 3)))
+
+
+def _gelu_d1(x):
+    th = np.tanh(_C * (x + 0.044715 * x ** 3))
+    du = _C * (1.0 + 3 * 0.044715 * x * x)
+    return 0.5 * (1.0 + th) + 0.5 * x * (1.0 - th * th) * du
+
+
+def _gelu_d2(x):
+    th = np.tanh(_C * (x + 0.044715 * x ** 3))
+    du = _C * (1.0 + 3 * 0.044715 * x * x)
+    d2u = _C * 6 * 0.044715 * x
+    return (1.0 - th * th) * (du + 0.5 * x * (d2u - 2.0 * th * du * du))
+
+
+def _mlp_chunk_forward(Q, X, V, e, W1, b1, W2, b2, gam, bet, eps):
+    n, d = X.shape
+    M = np.tril(np.ones((n, n)))
+    Z1 = X @ W1 + b1
+    Hh = _gelu(Z1)
+    Y = Hh @ W2 + b2
+    xh, s = _ln_rows(Y, eps)
+    R = X + gam * xh + bet - V
+    Gx = 2.0 * gam * R
+    m1 = Gx.mean(1, keepdims=True)
+    m2 = (Gx * xh).mean(1, keepdims=True)
+    G2 = s * (Gx - m1 - xh * m2)
+    U = G2 @ W2.T
+    G1 = U * _gelu_d1(Z1)
+    P = Q @ X.T
+    A = M * (e[None, :] * (P + 1.0))
+    Z1q = Q @ W1 + b1 - A @ G1
+    Hq = _gelu(Z1q)
+    P2 = Hq @ Hh.T
+    A2 = M * (e[None, :] * (P2 + 1.0))
+    Z2q = Hq @ W2 + b2 - A2 @ G2
+    zh, s2 = _ln_rows(Z2q, eps)
+    Z = Q + gam * zh + bet
+    new = (W1 - X.T @ (e[:, None] * G1), b1 - (e[:, None] * G1).sum(0),
+           W2 - Hh.T @ (e[:, None] * G2), b2 - (e[:, None] * G2).sum(0))
+    cache = dict(M=M, Z1=Z1, Hh=Hh, xh=xh, s=s, R=R, Gx=Gx, m1=m1, m2=m2, G2=G2, U=U, G1=G1, P=P, A=A,
+                 Z1q=Z1q, Hq=Hq, P2=P2, A2=A2, zh=zh, s2=s2, d=d)
+    return Z, new, cache
+
+
+def mlp_dual_form_backward(Q, K, V, eta, W1, b1, W2, b2, gam, bet, dZ, dS, chunk, eps=1e-6):
+    """TTT-MLP counterpart of dual_form_backward: gradients of sum(Z dZ) plus
+    the final state times dS = (dW1_T, db1_T, dW2_T, db2_T) for one (batch,
+    head).  Returns dQ, dK, dV, deta, dW1, db1, dW2, db2, dgam, dbet."""
+    T, d = Q.shape
+    starts = list(range(0, T, chunk))
+    states, S = [], (W1, b1, W2, b2)
+    for c0 in starts:
+        sl = slice(c0, c0 + chunk)
+        states.append(S)
+        _, S, _ = _mlp_chunk_forward(Q[sl], K[sl], V[sl], eta[sl], *S, gam, bet, eps)
+    dQ, dK, dV, de = (np.zeros_like(x) for x in (Q, K, V, eta))
+    dgam, dbet = np.zeros_like(gam), np.zeros_like(bet)
+    dW1n, db1n, dW2n, db2n = (x.copy() for x in dS)   # gradient of the state after the chunk
+    for c0, (cW1, cb1, cW2, cb2) in zip(reversed(starts), reversed(states)):
+        sl = slice(c0, c0 + chunk)
+        Qc, X, Vc, e = Q[sl], K[sl], V[sl], eta[sl]
+        _, _, k = _mlp_chunk_forward(Qc, X, Vc, e, cW1, cb1, cW2, cb2, gam, bet, eps)
+        M, G1, G2, Hh, Hq = k["M"], k["G1"], k["G2"], k["Hh"], k["Hq"]
+        dW1, db1, dW2, db2 = dW1n.copy(), db1n.copy(), dW2n.copy(), db2n.copy()
+        # output: z = q + gam z^ + bet, z^ = LN(Z2q)
+        dz = dZ[sl]
+        dgam += (dz * k["zh"]).sum(0)
+        dbet += dz.sum(0)
+        dQc = dz.copy()
+        dZ2q = _ln_back(dz * gam, k["zh"], k["s2"])
+        # Z2q = Hq W2 + b2 - A2 G2
+        dHq = dZ2q @ cW2.T
+        dW2 += Hq.T @ dZ2q
+        db2 += dZ2q.sum(0)
+        dA2 = -(dZ2q @ G2.T) * M
+        dG2 = -k["A2"].T @ dZ2q
+        # A2 = tril(eta_s (Hq Hh^T + 1))
+        de[sl] += (dA2 * (k["P2"] + 1.0)).sum(0)
+        dP2 = dA2 * e[None, :]
+        dHq += dP2 @ Hh
+        dHh = dP2.T @ Hq
+        # Hq = gelu(Z1q); Z1q = Q W1 + b1 - A G1
+        dZ1q = dHq * _gelu_d1(k["Z1q"])
+        dQc += dZ1q @ cW1.T
+        dW1 += Qc.T @ dZ1q
+        db1 += dZ1q.sum(0)
+        dA = -(dZ1q @ G1.T) * M
+        dG1 = -k["A"].T @ dZ1q
+        # A = tril(eta_s (Q X^T + 1))
+        de[sl] += (dA * (k["P"] + 1.0)).sum(0)
+        dP = dA * e[None, :]
+        dQc += dP @ X
+        dXc = dP.T @ Qc
+        # state update: W1' = W1 - X^T (eta G1), b1' = b1 - (eta G1)^T 1; the same for W2 with Hh, G2
+        dE1 = -(X @ dW1n) - db1n[None, :]
+        dG1 += e[:, None] * dE1
+        de[sl] += (dE1 * G1).sum(1)
+        dXc += -(e[:, None] * G1) @ dW1n.T
+        dE2 = -(Hh @ dW2n) - db2n[None, :]
+        dG2 += e[:, None] * dE2
+        de[sl] += (dE2 * G2).sum(1)
+        dHh += -(e[:, None] * G2) @ dW2n.T
+        # G1 = (G2 W2^T) * gelu'(Z1)
+        dU = dG1 * _gelu_d1(k["Z1"])
+        dZ1 = dG1 * k["U"] * _gelu_d2(k["Z1"])
+        dG2 += dU @ cW2
+        dW2 += dU.T @ G2
+        # G2 = LayerNorm backward of the reconstruction loss at Y
+        xh, s = k["xh"], k["s"]
+        mdg = (dG2 * xh).mean(1, keepdims=True)
+        dGx = s * (dG2 - dG2.mean(1, keepdims=True)) - s * mdg * xh
+        dxh = -s * k["m2"] * dG2 - s * mdg * k["Gx"]
+        ds = (dG2 * (k["Gx"] - k["m1"] - xh * k["m2"])).sum(1, keepdims=True)
+        dR = 2.0 * gam * dGx
+        dgam += (2.0 * k["R"] * dGx).sum(0) + (dR * xh).sum(0)
+        dbet += dR.sum(0)
+        dXc += dR
+        dV[sl] = -dR
+        dxh += gam * dR
+        dY = _ln_back(dxh, xh, s) - ds * s * s * xh / k["d"]
+        # Y = Hh W2 + b2; Hh = gelu(Z1); Z1 = X W1 + b1
+        dHh += dY @ cW2.T
+        dW2 += Hh.T @ dY
+        db2 += dY.sum(0)
+        dZ1 += dHh * _gelu_d1(k["Z1"])
+        dXc += dZ1 @ cW1.T
+        dW1 += X.T @ dZ1
+        db1 += dZ1.sum(0)
+        dQ[sl], dK[sl] = dQc, dXc
+        dW1n, db1n, dW2n, db2n = dW1, db1, dW2, db2
+    return dQ, dK, dV, de, dW1n, db1n, dW2n, db2n, dgam, dbet
+
+
+def mlp_case(seed, T, d=6, hid=10):
+    r = np.random.default_rng(seed)
+    Q, K, V = (r.normal(0, 1 / np.sqrt(d), (1, 1, T, d)) for _ in range(3))
+    eta = 1 / (1 + np.exp(-r.normal(0, 1, (1, 1, T)))) / d * 4
+    W1 = r.normal(0, 1 / np.sqrt(d), (1, 1, d, hid))
+    b1 = r.normal(0, 0.1, (1, 1, hid))
+    W2 = r.normal(0, 1 / np.sqrt(hid), (1, 1, hid, d))
+    b2 = r.normal(0, 0.1, (1, 1, d))
+    gamma = 1 + r.normal(0, 0.2, (1, d))
+    beta = r.normal(0, 0.2, (1, d))
+    dZ = r.normal(0, 1, (1, 1, T, d))
+    dS = (r.normal(0, 1, (1, 1, d, hid)), r.normal(0, 1, (1, 1, hid)), r.normal(0, 1, (1, 1, hid, d)),
+          r.normal(0, 1, (1, 1, d)))
+    return [Q, K, V, eta, W1, b1, W2, b2, gamma, beta], dZ, dS
+
+
+def test_gelu_derivatives_against_differences():
+    x = np.linspace(-4, 4, 81)
+    h = 1e-5
+    assert rel(_gelu_d1(x), (_gelu(x + h) - _gelu(x - h)) / (2 * h)) < 1e-8
+    assert rel(_gelu_d2(x), (_gelu_d1(x + h) - _gelu_d1(x - h)) / (2 * h)) < 1e-7
+
+
+@pytest.mark.parametrize("T,chunk", [(24, 8), (20, 8), (12, 4), (5, 1)])
+def test_mlp_chunked_backward_equals_the_oracle(T, chunk):
+    ins, dZ, dS = mlp_case(T + chunk, T)
+    ref = ob.ttt_mlp_backward(*ins, dZ, chunk, d_state=dS)
+    squeeze = lambda x: x[0, 0] if x.ndim >= 3 else x[0]
+    got = mlp_dual_form_backward(*(squeeze(x) for x in ins), squeeze(dZ), tuple(squeeze(x) for x in dS), chunk)
+    names = ("dQ", "dK", "dV", "deta", "dW1", "db1", "dW2", "db2", "dgamma", "dbeta")
+    for name, g, r in zip(names, got, ref):
+        assert rel(g, squeeze(r)) < 1e-10, f"{name}: {rel(g, squeeze(r)):.2e}"
