@@ -442,6 +442,30 @@ def test_float32_rounding_growth_is_inside_tolerance():
 # Regression fixture written by tests/golden/make_golden.py (oracle only)
 # ----------------------------------------------------------------------------
 
+def test_golden_regression_mlp_small():
+    g = read_golden("mlp_small_seed0.txt")
+    w = WORKLOADS["mlp_8k"].with_shape(B=1, H=1, T=48)
+    inp = make_inputs(w, 0)
+    keys = ("Q", "K", "V", "eta", "W1_0", "b1_0", "W2_0", "b2_0", "gamma", "beta")
+    Z, W1_T, b1_T, W2_T, b2_T = oracle.ttt_mlp(*(inp[k] for k in keys), w.mini_batch, w.ln_eps)
+    idx = g["Z_index"].astype(int)
+    np.testing.assert_allclose(Z.reshape(-1)[idx], g["Z"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(W2_T.reshape(-1)[:32], g["W2_T_head"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(b1_T.reshape(-1)[:16], g["b1_T_head"], rtol=1e-12, atol=1e-14)
+
+
+def test_golden_regression_linear_decode_pieces():
+    g = read_golden("linear_decode_pieces_seed0.txt")
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=1, T=40)
+    inp = make_inputs(w, 0)
+    cuts = [int(c) for c in g["cuts"]]
+    Z, _, _, W_mb, _ = decode_in_pieces(inp["Q"], inp["K"], inp["V"], inp["eta"], inp["W0"], inp["b0"],
+                                        inp["gamma"], inp["beta"], 16, cuts)
+    idx = g["Z_index"].astype(int)
+    np.testing.assert_allclose(Z.reshape(-1)[idx], g["Z"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(W_mb.reshape(-1)[:32], g["W_mb_head"], rtol=1e-12, atol=1e-14)
+
+
 def test_golden_regression_linear_tiny():
     g = read_golden("linear_tiny_f32_seed0.txt")
     w = WORKLOADS["linear_tiny_f32"]
@@ -452,10 +476,6 @@ def test_golden_regression_linear_tiny():
     np.testing.assert_allclose(Z.reshape(-1)[idx], g["Z"], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(W_T.reshape(-1)[:32], g["W_T_head"], rtol=1e-12, atol=1e-14)
 
-
-# ----------------------------------------------------------------------------
-# The pins catch plausible mistakes (mutations planted in a copy of the oracle)
-# ----------------------------------------------------------------------------
 
 # ----------------------------------------------------------------------------
 # Decode: the scan continued from the middle of a mini-batch (Key takeaways,
@@ -570,6 +590,10 @@ def test_mlp_decode_whole_stream_is_the_forward_scan():
     for a, b in zip(dec[:5], fwd):
         np.testing.assert_array_equal(a, b)
 
+
+# ----------------------------------------------------------------------------
+# The pins catch plausible mistakes (mutations planted in a copy of the oracle)
+# ----------------------------------------------------------------------------
 
 MUTATIONS = {
     "drop_mean_term": ("g[j] = s * (g[j] - mean_gx - xhat[j] * mean_gxx);",
