@@ -85,6 +85,8 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "ttt_linear_lag_kernel": ("ttt_linear_lag.cu", "ptx.cuh", "common.cuh", "tma_host.h", "ttt_internal.h"),
+    "ttt_linear_umma_kernel": ("ttt_linear_umma.cu", "ptx.cuh", "tcgen05.cuh", "common.cuh", "tma_host.h",
+                               "ttt_internal.h"),
     "ttt_linear_generic_kernel": ("ttt_linear_generic.cu", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_tc_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_split_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
@@ -519,7 +521,7 @@ def run_ours(args, world, rank, local):
     call(host_in)
     torch.cuda.synchronize(dev)
     dist_barrier(world)
-    e2e_steps = max(1, min(args.steps, 3))
+    e2e_steps = max(5, min(args.steps, 20))
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
         call(host_in)  # returns after the device->host copies finish
@@ -543,7 +545,8 @@ def run_ours(args, world, rank, local):
         else:
             family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
                 w.B, w.H, w.T, w.d, w.mini_batch, w.dtype, w.mode)
-            kname = {"tensorcore": "ttt_linear_lag_kernel", "generic": "ttt_linear_generic_kernel"}[family]
+            kname = {"tensorcore": "ttt_linear_lag_kernel", "tcgen05": "ttt_linear_umma_kernel",
+                     "generic": "ttt_linear_generic_kernel"}[family]
             achieved, peak, bound, unit = ab / (kernel_ms * 1e-3) / 1e9, hbm, "hbm", "GB/s"
         traffic = recorded_traffic(kname, w.name)
         line = {
@@ -575,13 +578,22 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
                     choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS])
-    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split", "tcgen05"],
+                    default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,
                     help="CPU seconds of oracle work per reference sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks with torchrun on this node
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", os.environ.get("MASTER_PORT", "29511"),
+               os.path.abspath(__file__), *sys.argv[1:]]
+        sys.exit(subprocess.call(cmd))
     world, rank, local = dist_setup()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks were started")
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)

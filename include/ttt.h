@@ -56,7 +56,17 @@
  *               environment variable TTT_CHECK=1 the call synchronises the
  *               stream after the launch and returns TTT_ERR_CUDA on an
  *               asynchronous error, or TTT_ERR_TIMEOUT if a kernel abandoned a
- *               bounded wait (its outputs are then undefined).
+ *               bounded wait (its outputs are then undefined).  The kernels
+ *               record an abandoned wait in an error word per process, not
+ *               per call: a checked call clears it before its launch, so its
+ *               status covers that call alone, but checked calls that overlap
+ *               on several streams may see each other's timeouts.  Both
+ *               environment variables are read once per process.
+ *   Fault injection  TTT_DEBUG_DROP_CHUNK=<c> (a test hook, read once per
+ *               process) makes the tensor-core TTT-Linear kernels skip the
+ *               loads of chunk c, so their bounded waits give up.  While it is
+ *               set every call runs as if TTT_CHECK=1 and such a call returns
+ *               TTT_ERR_TIMEOUT; leave it unset in normal use.
  *   Threads     Entry points are re-entrant.
  *   Continuation  Feeding W_T (b_T) back as W0 (b0) continues the sequence
  *               when the split falls on a mini-batch boundary (bit for bit in
@@ -66,6 +76,8 @@
  */
 #ifndef TTT_B200_TTT_H
 #define TTT_B200_TTT_H
+
+#include <stddef.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -83,7 +95,8 @@ typedef enum {
     TTT_ERR_ALIAS = 5,       /* an output overlaps an input other than as allowed  */
     TTT_ERR_UNSUPPORTED = 6, /* d, hidden, mode or implementation not built       */
     TTT_ERR_CUDA = 7,        /* CUDA launch or execution error                     */
-    TTT_ERR_TIMEOUT = 8      /* a kernel gave up a bounded wait (TTT_CHECK=1 only) */
+    TTT_ERR_TIMEOUT = 8,     /* a kernel gave up a bounded wait (TTT_CHECK=1 only) */
+    TTT_ERR_WORKSPACE = 9    /* workspace NULL or smaller than its size query returns */
 } ttt_status;
 
 typedef enum { TTT_BF16 = 0, TTT_F32 = 1 } ttt_dtype;
@@ -96,9 +109,14 @@ typedef enum {
     TTT_IMPL_GENERIC = 1,    /* fp32 SIMT scan: every supported shape, dtype and mode */
     TTT_IMPL_TENSORCORE = 2, /* tensor-core scan: bf16 Q/K/V, b = 16, T a multiple of 16;
                                 TTT-Linear d = 64 in LN mode, TTT-MLP d = 64, hidden = 256 */
-    TTT_IMPL_TENSORCORE_SPLIT = 3 /* TTT-MLP only, same shapes as TTT_IMPL_TENSORCORE: each
-                                     scan's hidden units split over the two CTAs of a
-                                     cluster (two SMs per scan) */
+    TTT_IMPL_TENSORCORE_SPLIT = 3, /* TTT-MLP only, same shapes as TTT_IMPL_TENSORCORE: each
+                                      scan's hidden units split over the two CTAs of a
+                                      cluster (two SMs per scan) */
+    TTT_IMPL_TCGEN05 = 4 /* TTT-Linear only, same shapes as TTT_IMPL_TENSORCORE: the products
+                            with the state run on the 5th-generation tensor cores (tcgen05,
+                            fp32 accumulators in tensor memory, one issuing thread), the
+                            sequential per-chunk chain on warp-level mma; the state is kept
+                            centred on its per-row means, which are added back to W_T, b_T */
 } ttt_impl;
 
 /*
@@ -226,6 +244,43 @@ ttt_status ttt_mlp_decode_impl(int B, int H, int T, int d, int hidden, int mini_
  * TTT_IMPL_TENSORCORE. */
 ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                            ttt_dtype qkv_dtype);
+
+/*
+ * TTT-Linear layer backward: the gradients an outer training loop needs
+ * (literature record, Key takeaways bullet 2: the outer loop trains the views
+ * theta_K, theta_V, theta_Q, the initial weights and the learning rate).
+ * Given the forward arguments of ttt_linear_forward and the upstream gradient
+ * dZ of its output (and, optionally, dW_T, db_T of its final state), returns
+ * the gradients of   sum(Z * dZ) + sum(W_T * dW_T) + sum(b_T * db_T)
+ * with respect to every forward input:
+ *   dQ, dK, dV   [B][H][T][d] fp32 (whatever qkv_dtype is)
+ *   deta         [B][H][T]
+ *   dW0, db0     [B][H][d][d], [B][H][d]
+ *   dgamma, dbeta [H][d], summed over the batch in a fixed order
+ *   dW_T, db_T   may be NULL (zero)
+ * Built for TTT_LN_RESIDUAL, d = 16, 32 or 64, mini_batch 1, 2, 4, 8 or 16,
+ * any T (TTT_ERR_UNSUPPORTED otherwise; TTT_PLAIN is not built).
+ * workspace    caller-owned device scratch of at least
+ *              ttt_linear_backward_workspace_size(B, H, T, d, mini_batch)
+ *              bytes (16-byte aligned), else TTT_ERR_WORKSPACE.  The call
+ *              first runs the forward scan and records there the state every
+ *              mini-batch starts from (d*d + d floats per mini-batch and
+ *              head), then sweeps the mini-batches in reverse, recomputing
+ *              each one's intermediates from its recorded state.  Its contents
+ *              are undefined afterwards; calls that may overlap need separate
+ *              workspaces.
+ * Outputs may not overlap each other, the inputs or the workspace
+ * (TTT_ERR_ALIAS).  Other conventions as ttt_linear_forward.
+ */
+size_t ttt_linear_backward_workspace_size(int B, int H, int T, int d, int mini_batch);
+
+ttt_status ttt_linear_backward(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                               ttt_mode mode, float ln_eps, const void* Q, const void* K,
+                               const void* V, const float* eta, const float* W0, const float* b0,
+                               const float* ln_gamma, const float* ln_beta, const float* dZ,
+                               const float* dW_T, const float* db_T, float* dQ, float* dK, float* dV,
+                               float* deta, float* dW0, float* db0, float* dgamma, float* dbeta,
+                               void* workspace, size_t workspace_bytes, ttt_stream_t stream);
 
 /* Static string naming a status code; never NULL. */
 const char* ttt_status_string(ttt_status status);

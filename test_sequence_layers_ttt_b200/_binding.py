@@ -13,6 +13,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from contextlib import nullcontext as _nullcontext
 from typing import Optional, Tuple
 
 import torch
@@ -22,10 +23,10 @@ LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
 
 TTT_BF16, TTT_F32 = 0, 1
 TTT_LN_RESIDUAL, TTT_PLAIN = 0, 1
-IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3}
-_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split"}
+IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3, "tcgen05": 4}
+_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split", 4: "tcgen05"}
 STATUS = ["TTT_OK", "TTT_ERR_NULL", "TTT_ERR_SHAPE", "TTT_ERR_DTYPE", "TTT_ERR_ALIGN",
-          "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT"]
+          "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT", "TTT_ERR_WORKSPACE"]
 
 
 class TTTError(RuntimeError):
@@ -63,6 +64,10 @@ lib.ttt_mlp_decode.restype = _I
 lib.ttt_mlp_decode.argtypes = [_I] * 8 + [_F] + [_P] * 15 + [_P]
 lib.ttt_mlp_decode_impl.restype = _I
 lib.ttt_mlp_decode_impl.argtypes = [_I] * 8 + [_F] + [_P] * 15 + [_I, _P]
+lib.ttt_linear_backward_workspace_size.restype = ctypes.c_size_t
+lib.ttt_linear_backward_workspace_size.argtypes = [_I] * 5
+lib.ttt_linear_backward.restype = _I
+lib.ttt_linear_backward.argtypes = [_I] * 7 + [_F] + [_P] * 20 + [ctypes.c_size_t, _P]
 
 
 def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
@@ -116,12 +121,26 @@ def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(handle)
 
 
-class _HostRoundTrip:
-    """Moves CPU inputs to the GPU and device outputs back (end-to-end path)."""
+def _launch_stream(device: torch.device, stream):
+    """The stream a call enqueues on, as a torch stream object."""
+    if stream is None:
+        return torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(getattr(stream, "cuda_stream", stream)), device=device)
 
-    def __init__(self, tensors):
+
+class _HostRoundTrip:
+    """Moves CPU inputs to the GPU and device outputs back (end-to-end path).
+
+    The copies in, the launch and the copies back are all enqueued on the one
+    stream the call launches on, so stream order alone makes the kernel see its
+    inputs and the copies back see its outputs."""
+
+    def __init__(self, tensors, stream=None):
         self.on_host = any(t is not None and t.device.type == "cpu" for t in tensors)
         self.device = torch.device("cuda", torch.cuda.current_device()) if self.on_host else None
+        self.stream = _launch_stream(self.device, stream) if self.on_host else None
 
     def to_device(self, t):
         if t is None or not self.on_host:
@@ -129,20 +148,22 @@ class _HostRoundTrip:
         if t.device.type != "cpu":
             return t
         src = t if t.is_pinned() else t.pin_memory()
-        return src.to(self.device, non_blocking=True)
+        with torch.cuda.stream(self.stream):
+            return src.to(self.device, non_blocking=True)
 
     def to_host(self, outs):
         if not self.on_host:
             return outs
         host = []
-        for o in outs:
-            if o is None:
-                host.append(None)
-                continue
-            h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-            h.copy_(o, non_blocking=True)
-            host.append(h)
-        torch.cuda.current_stream(self.device).synchronize()
+        with torch.cuda.stream(self.stream):
+            for o in outs:
+                if o is None:
+                    host.append(None)
+                    continue
+                h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+                h.copy_(o, non_blocking=True)
+                host.append(h)
+        self.stream.synchronize()
         return tuple(host)
 
 
@@ -223,7 +244,9 @@ def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *
         return _host_pipeline(run, dict(Q=Q, K=K, V=V, eta=eta, W0=W0, b0=b0),
                               dict(ln_gamma=ln_gamma, ln_beta=ln_beta),
                               dict(Z=(B, H, T, d), W_T=(B, H, d, d), b_T=None if plain else (B, H, d)))
-    rt = _HostRoundTrip([Q, K, V, eta, W0])
+    rt = _HostRoundTrip([Q, K, V, eta, W0], stream)
+    if rt.on_host:
+        stream = rt.stream
     Q, K, V, eta, W0, b0, ln_gamma, ln_beta = (
         rt.to_device(x) for x in (Q, K, V, eta, W0, b0, ln_gamma, ln_beta))
     B, H, T, d = Q.shape
@@ -237,12 +260,13 @@ def ttt_linear_forward(Q, K, V, eta, W0, b0=None, ln_gamma=None, ln_beta=None, *
     if tuple(eta.shape) != (B, H, T) or tuple(W0.shape) != (B, H, d, d):
         raise ValueError("eta must be [B,H,T] and W0 [B,H,d,d]")
     dev = Q.device
-    if Z is None:
-        Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
-    if W_T is None:
-        W_T = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
-    if b_T is None and m == TTT_LN_RESIDUAL:
-        b_T = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(rt.stream) if rt.on_host else _nullcontext():
+        if Z is None:
+            Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+        if W_T is None:
+            W_T = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+        if b_T is None and m == TTT_LN_RESIDUAL:
+            b_T = torch.empty((B, H, d), dtype=torch.float32, device=dev)
     st = lib.ttt_linear_forward_impl(
         B, H, T, d, int(mini_batch), _dtype_code(Q), m, float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
         _ptr(eta), _ptr(W0), _ptr(b0), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _ptr(W_T),
@@ -334,7 +358,9 @@ def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
                               dict(ln_gamma=ln_gamma, ln_beta=ln_beta),
                               dict(Z=(B, H, T, d), W1_T=(B, H, d, hid), b1_T=(B, H, hid),
                                    W2_T=(B, H, hid, d), b2_T=(B, H, d)))
-    rt = _HostRoundTrip([Q, K, V, eta, W1_0])
+    rt = _HostRoundTrip([Q, K, V, eta, W1_0], stream)
+    if rt.on_host:
+        stream = rt.stream
     Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta = (
         rt.to_device(x) for x in (Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta))
     B, H, T, d = Q.shape
@@ -345,11 +371,12 @@ def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
     dev = Q.device
     f32 = dict(dtype=torch.float32, device=dev)
-    Z = torch.empty((B, H, T, d), **f32) if Z is None else Z
-    W1_T = torch.empty((B, H, d, hid), **f32) if W1_T is None else W1_T
-    b1_T = torch.empty((B, H, hid), **f32) if b1_T is None else b1_T
-    W2_T = torch.empty((B, H, hid, d), **f32) if W2_T is None else W2_T
-    b2_T = torch.empty((B, H, d), **f32) if b2_T is None else b2_T
+    with torch.cuda.stream(rt.stream) if rt.on_host else _nullcontext():
+        Z = torch.empty((B, H, T, d), **f32) if Z is None else Z
+        W1_T = torch.empty((B, H, d, hid), **f32) if W1_T is None else W1_T
+        b1_T = torch.empty((B, H, hid), **f32) if b1_T is None else b1_T
+        W2_T = torch.empty((B, H, hid, d), **f32) if W2_T is None else W2_T
+        b2_T = torch.empty((B, H, d), **f32) if b2_T is None else b2_T
     st = lib.ttt_mlp_forward_impl(
         B, H, T, d, hid, int(mini_batch), _dtype_code(Q), float(ln_eps), _ptr(Q), _ptr(K),
         _ptr(V), _ptr(eta), _ptr(W1_0), _ptr(b1_0), _ptr(W2_0), _ptr(b2_0), _ptr(ln_gamma),
@@ -357,3 +384,45 @@ def ttt_mlp_forward(Q, K, V, eta, W1_0, b1_0, W2_0, b2_0, ln_gamma, ln_beta, *,
         _stream_handle(dev, stream))
     _check(st)
     return rt.to_host((Z, W1_T, b1_T, W2_T, b2_T))
+
+
+def linear_backward_workspace_size(B: int, H: int, T: int, d: int, mini_batch: int) -> int:
+    """Bytes of device workspace ttt_linear_backward needs (see include/ttt.h)."""
+    return int(lib.ttt_linear_backward_workspace_size(B, H, T, d, mini_batch))
+
+
+def ttt_linear_backward(Q, K, V, eta, W0, b0, ln_gamma, ln_beta, dZ, dW_T=None, db_T=None, *,
+                        mini_batch: int = 16, mode="ln", ln_eps: float = 1e-6, workspace=None, stream=None):
+    """TTT-Linear layer backward (see include/ttt.h): gradients of
+    sum(Z dZ) + sum(W_T dW_T) + sum(b_T db_T) with respect to the forward inputs.
+    Returns (dQ, dK, dV, deta, dW0, db0, dgamma, dbeta), fp32 CUDA tensors.  The
+    workspace (a CUDA byte tensor) is allocated here when not given."""
+    B, H, T, d = Q.shape
+    named = (("Q", Q), ("K", K), ("V", V), ("eta", eta), ("W0", W0), ("b0", b0), ("ln_gamma", ln_gamma),
+             ("ln_beta", ln_beta), ("dZ", dZ), ("dW_T", dW_T), ("db_T", db_T))
+    for name, t in named:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if K.shape != Q.shape or V.shape != Q.shape or K.dtype != Q.dtype or V.dtype != Q.dtype:
+        raise ValueError("Q, K, V must share shape and dtype")
+    if tuple(dZ.shape) != (B, H, T, d) or dZ.dtype != torch.float32:
+        raise ValueError("dZ must be float32 [B,H,T,d]")
+    dev = Q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty((B, H, T, d), **f32) for _ in range(3))
+    deta = torch.empty((B, H, T), **f32)
+    dW0 = torch.empty((B, H, d, d), **f32)
+    db0 = torch.empty((B, H, d), **f32)
+    dgamma = torch.empty((H, d), **f32)
+    dbeta = torch.empty((H, d), **f32)
+    need = linear_backward_workspace_size(B, H, T, d, mini_batch)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib.ttt_linear_backward(
+        B, H, T, d, int(mini_batch), _dtype_code(Q), _mode_code(mode), float(ln_eps), _ptr(Q), _ptr(K), _ptr(V),
+        _ptr(eta), _ptr(W0), _ptr(b0), _ptr(ln_gamma), _ptr(ln_beta), _ptr(dZ), _ptr(dW_T), _ptr(db_T),
+        _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0), _ptr(db0), _ptr(dgamma), _ptr(dbeta),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        _stream_handle(dev, stream))
+    _check(st)
+    return dQ, dK, dV, deta, dW0, db0, dgamma, dbeta

@@ -34,8 +34,23 @@ bool overlap(Span a, Span b) {
 }
 
 bool check_env() {
-    const char* v = std::getenv("TTT_CHECK");
-    return v && v[0] && std::strcmp(v, "0") != 0;
+    static const bool on = [] {
+        const char* v = std::getenv("TTT_CHECK");
+        return v && v[0] && std::strcmp(v, "0") != 0;
+    }();
+    // the fault-injection hook makes a launch abandon its waits: report that as a status
+    return on || ttt::drop_chunk_hook() >= 0;
+}
+
+// In check mode the device error words are cleared before the launch, so the
+// status a checked call returns reflects that call alone (calls overlapping on
+// several streams still share the words).
+bool prepare() {
+    if (!check_env()) return true;
+    unsigned int stale = 0;
+    return ttt::read_and_clear_device_error(&stale) == cudaSuccess &&
+           ttt::read_and_clear_mlp_error(&stale) == cudaSuccess &&
+           ttt::read_and_clear_umma_error(&stale) == cudaSuccess;
 }
 
 bool valid_mini_batch(int mb) { return mb >= 1 && (mb % 16 == 0 || mb == 1 || mb == 2 || mb == 4 || mb == 8); }
@@ -58,10 +73,11 @@ ttt_status finish(cudaError_t launch, cudaStream_t stream) {
     if (launch != cudaSuccess) return TTT_ERR_CUDA;
     if (!check_env()) return TTT_OK;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
-    unsigned int flag = 0, mlp_flag = 0;
+    unsigned int flag = 0, mlp_flag = 0, umma_flag = 0;
     if (ttt::read_and_clear_device_error(&flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_mlp_error(&mlp_flag) != cudaSuccess) return TTT_ERR_CUDA;
-    return (flag | mlp_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
+    if (ttt::read_and_clear_umma_error(&umma_flag) != cudaSuccess) return TTT_ERR_CUDA;
+    return (flag | mlp_flag | umma_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
 }
 
 ttt_status validate_linear(const LinearArgs& a) {
@@ -157,9 +173,74 @@ ttt_status validate_mlp_decode(const MlpArgs& a) {
     return check_aliasing(outs, 9, ins, same_as, 6);
 }
 
+// Layer backward: shapes and modes the backward kernels take, pointers, alignment,
+// workspace size and overlaps (every output is distinct from every input, from
+// the workspace and from every other output).
+ttt_status validate_linear_backward(const ttt::LinearBwdArgs& a, const void* workspace, size_t workspace_bytes) {
+    const LinearArgs& f = a.f;
+    if (f.B < 1 || f.H < 1 || f.T < 0 || (long long)f.B * f.H > INT_MAX) return TTT_ERR_SHAPE;
+    if (!valid_mini_batch(f.mini_batch)) return TTT_ERR_SHAPE;
+    if (f.dtype != TTT_BF16 && f.dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (f.mode != TTT_LN_RESIDUAL && f.mode != TTT_PLAIN) return TTT_ERR_UNSUPPORTED;
+    if (!(f.ln_eps > 0.f)) return TTT_ERR_SHAPE;
+    if (!ttt::linear_backward_supports(a)) return TTT_ERR_UNSUPPORTED;
+    if (f.T > 0 && (!f.Q || !f.K || !f.V || !f.eta || !a.dZ || !a.dQ || !a.dK || !a.dV || !a.deta))
+        return TTT_ERR_NULL;
+    if (!f.W0 || !f.b0 || !f.gamma || !f.beta || !a.dW0 || !a.db0 || !a.dgamma || !a.dbeta) return TTT_ERR_NULL;
+    const void* ptrs[] = {f.Q, f.K, f.V, f.eta, f.W0, f.b0, f.gamma, f.beta, a.dZ, a.dW_T, a.db_T, a.dQ,
+                          a.dK, a.dV, a.deta, a.dW0, a.db0, a.dgamma, a.dbeta, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TTT_ERR_ALIGN;
+    const size_t need = ttt::linear_backward_workspace_bytes(f.B, f.H, f.T, f.d, f.mini_batch);
+    if (!workspace || workspace_bytes < need) return TTT_ERR_WORKSPACE;
+    const size_t es = f.dtype == TTT_BF16 ? 2 : 4;
+    const size_t bh = (size_t)f.B * f.H, ntok = bh * (size_t)f.T, d = f.d;
+    Span ins[] = {{f.Q, ntok * d * es},      {f.K, ntok * d * es},         {f.V, ntok * d * es},
+                  {f.eta, ntok * 4},         {f.W0, bh * d * d * 4},       {f.b0, bh * d * 4},
+                  {f.gamma, (size_t)f.H * d * 4}, {f.beta, (size_t)f.H * d * 4}, {a.dZ, ntok * d * 4},
+                  {a.dW_T, a.dW_T ? bh * d * d * 4 : 0}, {a.db_T, a.db_T ? bh * d * 4 : 0}, {workspace, need}};
+    Span outs[] = {{a.dQ, ntok * d * 4}, {a.dK, ntok * d * 4},   {a.dV, ntok * d * 4},
+                   {a.deta, ntok * 4},   {a.dW0, bh * d * d * 4}, {a.db0, bh * d * 4},
+                   {a.dgamma, (size_t)f.H * d * 4}, {a.dbeta, (size_t)f.H * d * 4}};
+    const int same_as[] = {-1, -1, -1, -1, -1, -1, -1, -1};
+    return check_aliasing(outs, 8, ins, same_as, 12);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t ttt_linear_backward_workspace_size(int B, int H, int T, int d, int mini_batch) {
+    return ttt::linear_backward_workspace_bytes(B, H, T, d, mini_batch);
+}
+
+ttt_status ttt_linear_backward(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype, ttt_mode mode,
+                               float ln_eps, const void* Q, const void* K, const void* V, const float* eta,
+                               const float* W0, const float* b0, const float* ln_gamma, const float* ln_beta,
+                               const float* dZ, const float* dW_T, const float* db_T, float* dQ, float* dK,
+                               float* dV, float* deta, float* dW0, float* db0, float* dgamma, float* dbeta,
+                               void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+    ttt::LinearBwdArgs a{};
+    a.f = LinearArgs{B, H, T, d, mini_batch, qkv_dtype, mode, ln_eps, Q, K, V, eta, W0, b0, ln_gamma, ln_beta,
+                     nullptr, nullptr, nullptr};
+    a.dZ = dZ;
+    a.dW_T = dW_T;
+    a.db_T = db_T;
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.deta = deta;
+    a.dW0 = dW0;
+    a.db0 = db0;
+    a.dgamma = dgamma;
+    a.dbeta = dbeta;
+    ttt_status st = validate_linear_backward(a, workspace, workspace_bytes);
+    if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return finish(ttt::launch_linear_backward(a, static_cast<float*>(workspace), s), s);
+}
+
 
 ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
                                    ttt_mode mode, float ln_eps, const void* Q, const void* K,
@@ -171,6 +252,7 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, t
                  W0, b0, ln_gamma, ln_beta, Z, W_T, b_T};
     ttt_status st = validate_linear(a);
     if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (impl) {
         case TTT_IMPL_AUTO:
@@ -181,6 +263,9 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, t
         case TTT_IMPL_TENSORCORE:
             if (!ttt::linear_tc_supports(a)) return TTT_ERR_UNSUPPORTED;
             return finish(ttt::launch_linear_tc(a, s), s);
+        case TTT_IMPL_TCGEN05:
+            if (!ttt::linear_umma_supports(a)) return TTT_ERR_UNSUPPORTED;
+            return finish(ttt::launch_linear_umma(a, s), s);
         default:
             return TTT_ERR_UNSUPPORTED;
     }
@@ -220,6 +305,7 @@ ttt_status ttt_linear_decode(int B, int H, int T, int d, int mini_batch, int pos
                  pos0, pos0 > 0 ? W_mb : nullptr, (pos0 > 0 && ln) ? b_mb : nullptr, W_mb, ln ? b_mb : nullptr};
     ttt_status st = validate_decode(a);
     if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (ttt::linear_decode_supports(a)) return finish(ttt::launch_linear_decode(a, s), s);
     return finish(ttt::launch_linear_generic(a, s), s);
@@ -235,6 +321,7 @@ ttt_status ttt_mlp_forward_impl(int B, int H, int T, int d, int hidden, int mini
               W2_0, b2_0, ln_gamma, ln_beta, Z, W1_T, b1_T, W2_T, b2_T};
     ttt_status st = validate_mlp(a);
     if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (impl == TTT_IMPL_AUTO) impl = mlp_auto_impl(a);
     switch (impl) {
@@ -260,6 +347,7 @@ ttt_status ttt_mlp_decode_impl(int B, int H, int T, int d, int hidden, int mini_
               ln_gamma, ln_beta, Z, W1, b1, W2, b2, pos0, W1_mb, b1_mb, W2_mb, b2_mb};
     ttt_status st = validate_mlp_decode(a);
     if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (impl) {
         case TTT_IMPL_AUTO:
@@ -310,10 +398,11 @@ const char* ttt_status_string(ttt_status status) {
         case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED: shape, mode or kernel family not built";
         case TTT_ERR_CUDA: return "TTT_ERR_CUDA: CUDA launch or execution error";
         case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+        case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE: workspace missing or smaller than required";
         default: return "TTT_ERR_UNKNOWN";
     }
 }
 
-int ttt_abi_version(void) { return 101; }
+int ttt_abi_version(void) { return 102; }
 
 }  // extern "C"

@@ -42,9 +42,25 @@ cudaError_t launch_linear_generic(const LinearArgs& a, cudaStream_t stream);
 bool linear_tc_supports(const LinearArgs& a);
 cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream);
 
+// State products on tcgen05 / TMEM, chain on mma.sync (ttt_linear_umma.cu); same shapes as linear_tc.
+bool linear_umma_supports(const LinearArgs& a);
+cudaError_t launch_linear_umma(const LinearArgs& a, cudaStream_t stream);
+cudaError_t read_and_clear_umma_error(unsigned int* out);
+
 // Decode with the state in registers (d = 64); in place on W_T / b_T and Wm_T / bm_T.
 bool linear_decode_supports(const LinearArgs& a);
 cudaError_t launch_linear_decode(const LinearArgs& a, cudaStream_t stream);
+
+// TTT-Linear layer backward (ttt_linear_backward.cu): the forward arguments plus
+// the upstream gradients and the gradient outputs.
+struct LinearBwdArgs {
+    LinearArgs f;  // Q, K, V, eta, W0, b0, gamma, beta and the shapes (Z, W_T, b_T unused)
+    const float *dZ, *dW_T, *db_T;
+    float *dQ, *dK, *dV, *deta, *dW0, *db0, *dgamma, *dbeta;
+};
+bool linear_backward_supports(const LinearBwdArgs& a);
+size_t linear_backward_workspace_bytes(int B, int H, int T, int d, int mini_batch);
+cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cudaStream_t stream);
 
 bool mlp_generic_supports(const MlpArgs& a);
 cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);
@@ -63,5 +79,9 @@ cudaError_t read_and_clear_mlp_error(unsigned int* out);
 
 // Device-side error word set by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_device_error(unsigned int* out);
+
+// Fault-injection hook: the chunk index named by TTT_DEBUG_DROP_CHUNK (read once
+// per process), whose loads the tensor-core TTT-Linear producer skips; -1 when unset.
+int drop_chunk_hook();
 
 }  // namespace ttt

@@ -1,0 +1,478 @@
+// TTT-Linear layer backward: the gradients an outer training loop needs
+// ("Learning to (Learn at Test Time)", literature record, Key takeaways
+// bullet 2: the outer loop trains the views theta_K, theta_V, theta_Q, the
+// initial weights and the learning rate), for the scan of bullets 1 and 5
+// with f(x) = x + LN(x W + b).
+//
+// Given upstream gradients dZ (and optionally dW_T, db_T of the final state),
+// computes the gradients of  sum(Z dZ) + sum(W_T dW_T) + sum(b_T db_T)  with
+// respect to Q, K, V, eta, W0, b0, gamma and beta.
+//
+// Two passes, one CTA per (batch, head), fp32 in shared memory:
+//   1. ttt_linear_states_kernel runs the forward scan mini-batch by mini-batch
+//      and records the state each mini-batch starts from, W_j (d x d) and b_j,
+//      in the caller's workspace (d^2 + d floats per mini-batch and head).
+//   2. ttt_linear_backward_kernel walks the mini-batches in reverse.  For each
+//      it reloads W_j, b_j, recomputes the mini-batch's intermediates
+//        Y = X W + b,  x^ = LN0(Y),  R = X + gamma x^ + beta - V,
+//        Gx = 2 gamma R,  G = s (Gx - mean Gx - x^ mean(Gx x^))   (= dl/dY)
+//        P = Q X^T,  A = tril(eta_s (P + 1)),  Zb = Q W + b - A G,  z^ = LN0(Zb)
+//      and applies the adjoint of each step, carrying dW, db (the gradient of
+//      the state after the mini-batch) backwards.  The LayerNorm backward that
+//      forms G is differentiated through, including the explicit dependence of
+//      G on s = (var Y + eps)^(-1/2).
+//   3. ttt_linear_dgamma_kernel sums the per-(batch, head) gamma / beta
+//      partials over the batch in a fixed order (deterministic).
+// One mini-batch is processed at a time (mini_batch <= 16 tokens).
+#include "common.cuh"
+#include "ttt_internal.h"
+
+namespace ttt {
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr int kMaxD = 64, kMaxN = 16;
+constexpr int LD = kMaxD + 1;  // padded row length of every [rows][d] array
+
+template <typename T>
+__device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i]); }
+
+// C (=|+=) alpha * op(A) op(B), op(A)(i,k) = TA ? A[k][i] : A[i][k], op(B)(k,j) = TB ? B[j][k] : B[k][j]
+template <bool TA, bool TB>
+__device__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+                    float alpha, bool accumulate) {
+    for (int idx = threadIdx.x; idx < M * N; idx += blockDim.x) {
+        const int i = idx / N, j = idx % N;
+        float acc = 0.f;
+        for (int k = 0; k < K; k++)
+            acc = fmaf(TA ? A[k * lda + i] : A[i * lda + k], TB ? B[j * ldb + k] : B[k * ldb + j], acc);
+        C[i * ldc + j] = accumulate ? fmaf(alpha, acc, C[i * ldc + j]) : alpha * acc;
+    }
+}
+
+struct BwdSmem {
+    float W[kMaxD * LD], b[kMaxD];         // state at the start of the mini-batch
+    float dW[kMaxD * LD], db[kMaxD];       // gradient of the state after it
+    float dWp[kMaxD * LD], dbp[kMaxD];     // gradient of the state before it
+    float X[kMaxN * LD], Qm[kMaxN * LD], Vm[kMaxN * LD], dZ[kMaxN * LD];
+    float xh[kMaxN * LD], R[kMaxN * LD], Gx[kMaxN * LD], G[kMaxN * LD], zh[kMaxN * LD];
+    float dZb[kMaxN * LD], dG[kMaxN * LD], dQc[kMaxN * LD], dXc[kMaxN * LD], tmp[kMaxN * LD];
+    float P[kMaxN * kMaxN], A[kMaxN * kMaxN], dA[kMaxN * kMaxN];
+    float s[kMaxN], s2[kMaxN], m1[kMaxN], m2[kMaxN], mdg[kMaxN], ds[kMaxN], e[kMaxN], de[kMaxN];
+    float gam[kMaxD], bet[kMaxD], dgam[kMaxD], dbet[kMaxD];
+};
+
+// x^ = (y - mean y) s, s = (var y + eps)^(-1/2), per row of y [n][d]; one warp per row
+__device__ void ln_rows(const float* y, float* xh, float* s, int n, int d, float eps) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int t = warp; t < n; t += nw) {
+        float a = 0.f;
+        for (int j = lane; j < d; j += 32) a += y[t * LD + j];
+        const float mu = warp_sum(a) / d;
+        float v = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            const float c = y[t * LD + j] - mu;
+            v = fmaf(c, c, v);
+        }
+        const float rs = rsqrtf(warp_sum(v) / d + eps);
+        for (int j = lane; j < d; j += 32) xh[t * LD + j] = (y[t * LD + j] - mu) * rs;
+        if (lane == 0) s[t] = rs;
+    }
+}
+
+// dy = s (dx^ - mean dx^ - x^ mean(dx^ x^)) per row, in place on dxh
+__device__ void ln_back_rows(float* dxh, const float* xh, const float* s, int n, int d) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int t = warp; t < n; t += nw) {
+        float a = 0.f, c = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            a += dxh[t * LD + j];
+            c = fmaf(dxh[t * LD + j], xh[t * LD + j], c);
+        }
+        const float ma = warp_sum(a) / d, mc = warp_sum(c) / d;
+        for (int j = lane; j < d; j += 32) dxh[t * LD + j] = s[t] * (dxh[t * LD + j] - ma - xh[t * LD + j] * mc);
+    }
+}
+
+// Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G)
+__device__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
+    bmm<false, false>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
+    __syncthreads();
+    ln_rows(m.tmp, m.xh, m.s, n, d, eps);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+        const int t = i / d, j = i % d, o = t * LD + j;
+        m.R[o] = m.X[o] + m.gam[j] * m.xh[o] + m.bet[j] - m.Vm[o];
+        m.Gx[o] = 2.f * m.gam[j] * m.R[o];
+    }
+    __syncthreads();
+    {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+        for (int t = warp; t < n; t += nw) {
+            float a = 0.f, c = 0.f;
+            for (int j = lane; j < d; j += 32) {
+                a += m.Gx[t * LD + j];
+                c = fmaf(m.Gx[t * LD + j], m.xh[t * LD + j], c);
+            }
+            a = warp_sum(a) / d;
+            c = warp_sum(c) / d;
+            if (lane == 0) {
+                m.m1[t] = a;
+                m.m2[t] = c;
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+        const int t = i / d, o = t * LD + i % d;
+        m.G[o] = m.s[t] * (m.Gx[o] - m.m1[t] - m.xh[o] * m.m2[t]);
+    }
+    __syncthreads();
+}
+
+template <typename T>
+__device__ void load_tokens(BwdSmem& m, const T* Q, const T* K, const T* V, const float* eta, size_t base, int n,
+                            int d) {
+    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+        const int t = i / d, j = i % d;
+        const size_t gi = base * d + i;
+        m.X[t * LD + j] = ldv(K, gi);
+        m.Qm[t * LD + j] = ldv(Q, gi);
+        m.Vm[t * LD + j] = ldv(V, gi);
+    }
+    for (int t = threadIdx.x; t < n; t += blockDim.x) m.e[t] = eta[base + t];
+}
+
+// ------------------------------------------------------------------ pass 1: states
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+ttt_linear_states_kernel(int T_, int d, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
+                         const float* W0, const float* b0, const float* gamma, const float* beta, int H,
+                         float* states) {
+    extern __shared__ float smem_f[];
+    BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
+    const int bh = blockIdx.x, h = bh % H;
+    const int nmb = (T_ + mb - 1) / mb;
+    const size_t sz = (size_t)d * d + d;
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) m.W[(i / d) * LD + i % d] = W0[(size_t)bh * d * d + i];
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        m.b[j] = b0[(size_t)bh * d + j];
+        m.gam[j] = gamma[h * d + j];
+        m.bet[j] = beta[h * d + j];
+    }
+    __syncthreads();
+    for (int jb = 0; jb < nmb; jb++) {
+        const int t0 = jb * mb, n = min(mb, T_ - t0);
+        float* st = states + ((size_t)bh * nmb + jb) * sz;
+        for (int i = threadIdx.x; i < d * d; i += blockDim.x) st[i] = m.W[(i / d) * LD + i % d];
+        for (int j = threadIdx.x; j < d; j += blockDim.x) st[d * d + j] = m.b[j];
+        load_tokens(m, Q, K, V, eta, (size_t)bh * T_ + t0, n, d);
+        __syncthreads();
+        chunk_inner_grad(m, n, d, eps);
+        // W -= X^T diag(e) G, b -= G^T e
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, o = t * LD + i % d;
+            m.tmp[o] = m.e[t] * m.G[o];
+        }
+        __syncthreads();
+        bmm<true, false>(m.W, LD, m.X, LD, m.tmp, LD, d, d, n, -1.f, true);
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float a = 0.f;
+            for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
+            m.b[j] -= a;
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ pass 2: the reverse sweep
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+ttt_linear_backward_kernel(int T_, int d, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
+                           const float* gamma, const float* beta, int H, const float* states, const float* dZ,
+                           const float* dW_T, const float* db_T, float* dQ, float* dK, float* dV, float* deta,
+                           float* dW0, float* db0, float* gb_partial) {
+    extern __shared__ float smem_f[];
+    BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
+    const int bh = blockIdx.x, h = bh % H;
+    const int nmb = (T_ + mb - 1) / mb;
+    const size_t sz = (size_t)d * d + d;
+    const float inv_d = 1.f / d;
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x)
+        m.dW[(i / d) * LD + i % d] = dW_T ? dW_T[(size_t)bh * d * d + i] : 0.f;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        m.db[j] = db_T ? db_T[(size_t)bh * d + j] : 0.f;
+        m.gam[j] = gamma[h * d + j];
+        m.bet[j] = beta[h * d + j];
+        m.dgam[j] = 0.f;
+        m.dbet[j] = 0.f;
+    }
+    __syncthreads();
+    for (int jb = nmb - 1; jb >= 0; jb--) {
+        const int t0 = jb * mb, n = min(mb, T_ - t0);
+        const size_t base = (size_t)bh * T_ + t0;
+        const float* st = states + ((size_t)bh * nmb + jb) * sz;
+        for (int i = threadIdx.x; i < d * d; i += blockDim.x) m.W[(i / d) * LD + i % d] = st[i];
+        for (int j = threadIdx.x; j < d; j += blockDim.x) m.b[j] = st[d * d + j];
+        load_tokens(m, Q, K, V, eta, base, n, d);
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.dZ[(i / d) * LD + i % d] = dZ[base * d + i];
+        __syncthreads();
+        // ---- recompute the mini-batch's forward
+        chunk_inner_grad(m, n, d, eps);
+        bmm<false, true>(m.P, kMaxN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
+            const int t = i / n, s_ = i % n;
+            m.A[t * kMaxN + s_] = s_ <= t ? m.e[s_] * (m.P[t * kMaxN + s_] + 1.f) : 0.f;
+        }
+        __syncthreads();
+        // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb)
+        bmm<false, false>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false);
+        __syncthreads();
+        bmm<false, false>(m.tmp, LD, m.A, kMaxN, m.G, LD, n, d, n, -1.f, true);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
+        __syncthreads();
+        ln_rows(m.tmp, m.zh, m.s2, n, d, eps);
+        __syncthreads();
+        // ---- z = q + gamma z^ + beta
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float a = 0.f, c = 0.f;
+            for (int t = 0; t < n; t++) {
+                a = fmaf(m.dZ[t * LD + j], m.zh[t * LD + j], a);
+                c += m.dZ[t * LD + j];
+            }
+            m.dgam[j] += a;
+            m.dbet[j] += c;
+        }
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int o = (i / d) * LD + i % d;
+            m.dQc[o] = m.dZ[o];
+            m.dZb[o] = m.dZ[o] * m.gam[i % d];
+        }
+        __syncthreads();
+        ln_back_rows(m.dZb, m.zh, m.s2, n, d);
+        __syncthreads();
+        // ---- Zb = Q W + b - A G
+        bmm<false, true>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true);      // dQ += dZb W^T
+        bmm<true, false>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);    // dW_prev = Q^T dZb
+        bmm<false, true>(m.dA, kMaxN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
+        bmm<true, false>(m.dG, LD, m.A, kMaxN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float a = 0.f;
+            for (int t = 0; t < n; t++) a += m.dZb[t * LD + j];
+            m.dbp[j] = a + m.db[j];
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
+            const int t = i / n, s_ = i % n;
+            if (s_ > t) m.dA[t * kMaxN + s_] = 0.f;
+        }
+        // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp)
+        bmm<false, false>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, j = i % d, o = t * LD + j;
+            m.tmp[o] -= m.db[j];
+            m.dG[o] = fmaf(m.e[t], m.tmp[o], m.dG[o]);
+        }
+        __syncthreads();
+        {
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+            for (int t = warp; t < n; t += nw) {  // de = sum_j dEG G + sum_t dA (P + 1)
+                float a = 0.f;
+                for (int j = lane; j < d; j += 32) a = fmaf(m.tmp[t * LD + j], m.G[t * LD + j], a);
+                a = warp_sum(a);
+                float c = 0.f;
+                for (int r = lane; r < n; r += 32) c = fmaf(m.dA[r * kMaxN + t], m.P[r * kMaxN + t] + 1.f, c);
+                c = warp_sum(c);
+                if (lane == 0) m.de[t] = a + c;
+            }
+        }
+        __syncthreads();  // tmp is read above and overwritten below
+        // dX = -(e G) dW^T  (tmp <- e G)
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, o = t * LD + i % d;
+            m.tmp[o] = m.e[t] * m.G[o];
+        }
+        __syncthreads();
+        bmm<false, true>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false);
+        // dW_prev += dW (the state passes through)
+        for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
+            const int o = (i / d) * LD + i % d;
+            m.dWp[o] += m.dW[o];
+        }
+        // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
+        for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * kMaxN + i % n] *= m.e[i % n];
+        __syncthreads();
+        bmm<false, false>(m.dQc, LD, m.dA, kMaxN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
+        bmm<true, false>(m.dXc, LD, m.dA, kMaxN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
+        // ---- G = s (Gx - m1 - x^ m2), Gx = 2 gamma R, R = X + gamma x^ + beta - V
+        {
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+            for (int t = warp; t < n; t += nw) {
+                float a = 0.f, c = 0.f, e2 = 0.f;
+                for (int j = lane; j < d; j += 32) {
+                    const int o = t * LD + j;
+                    a = fmaf(m.dG[o], m.xh[o], a);
+                    c += m.dG[o];
+                    e2 = fmaf(m.dG[o], m.Gx[o] - m.m1[t] - m.xh[o] * m.m2[t], e2);
+                }
+                a = warp_sum(a) * inv_d;
+                c = warp_sum(c) * inv_d;
+                e2 = warp_sum(e2);
+                if (lane == 0) {
+                    m.mdg[t] = a;
+                    m.m1[t] = c;  // m1 is no longer needed: reuse it for mean(dG)
+                    m.ds[t] = e2;
+                }
+            }
+        }
+        __syncthreads();
+        // dGx (into dZb), dxh (into tmp), dR (into dG)
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, j = i % d, o = t * LD + j;
+            const float s_ = m.s[t];
+            const float dgx = s_ * (m.dG[o] - m.m1[t]) - s_ * m.mdg[t] * m.xh[o];
+            const float dxh = -s_ * m.m2[t] * m.dG[o] - s_ * m.mdg[t] * m.Gx[o];
+            const float dr = 2.f * m.gam[j] * dgx;
+            m.dZb[o] = dgx;
+            m.tmp[o] = dxh + m.gam[j] * dr;
+            m.dG[o] = dr;
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float a = 0.f, c = 0.f;
+            for (int t = 0; t < n; t++) {
+                const int o = t * LD + j;
+                a += 2.f * m.R[o] * m.dZb[o] + m.dG[o] * m.xh[o];
+                c += m.dG[o];
+            }
+            m.dgam[j] += a;
+            m.dbet[j] += c;
+        }
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, j = i % d, o = t * LD + j;
+            m.dXc[o] += m.dG[o];
+            dV[(base + t) * d + j] = -m.dG[o];
+        }
+        __syncthreads();
+        // x^ = LN0(Y), and s appears explicitly in G: dY = LNback(dxh) - ds s^2 x^ / d  (into tmp)
+        ln_back_rows(m.tmp, m.xh, m.s, n, d);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, o = t * LD + i % d;
+            m.tmp[o] -= m.ds[t] * m.s[t] * m.s[t] * m.xh[o] * inv_d;
+        }
+        __syncthreads();
+        // ---- Y = X W + b
+        bmm<false, true>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true);     // dX += dY W^T
+        bmm<true, false>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true);     // dW_prev += X^T dY
+        for (int j = threadIdx.x; j < d; j += blockDim.x) {
+            float a = 0.f;
+            for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
+            m.dbp[j] += a;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
+            const int t = i / d, j = i % d, o = t * LD + j;
+            dQ[(base + t) * d + j] = m.dQc[o];
+            dK[(base + t) * d + j] = m.dXc[o];
+        }
+        for (int t = threadIdx.x; t < n; t += blockDim.x) deta[base + t] = m.de[t];
+        for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
+            const int o = (i / d) * LD + i % d;
+            m.dW[o] = m.dWp[o];
+        }
+        for (int j = threadIdx.x; j < d; j += blockDim.x) m.db[j] = m.dbp[j];
+        __syncthreads();
+    }
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) dW0[(size_t)bh * d * d + i] = m.dW[(i / d) * LD + i % d];
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        db0[(size_t)bh * d + j] = m.db[j];
+        gb_partial[((size_t)bh * 2 + 0) * d + j] = m.dgam[j];
+        gb_partial[((size_t)bh * 2 + 1) * d + j] = m.dbet[j];
+    }
+}
+
+// ------------------------------------------------------------------ pass 3: gamma / beta over the batch
+__global__ void ttt_linear_dgamma_kernel(int B, int H, int d, const float* gb_partial, float* dgamma, float* dbeta) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= H * d) return;
+    const int h = i / d, j = i % d;
+    float a = 0.f, c = 0.f;
+    for (int b = 0; b < B; b++) {
+        const size_t bh = (size_t)b * H + h;
+        a += gb_partial[(bh * 2 + 0) * d + j];
+        c += gb_partial[(bh * 2 + 1) * d + j];
+    }
+    dgamma[i] = a;
+    dbeta[i] = c;
+}
+
+}  // namespace
+
+bool linear_backward_supports(const LinearBwdArgs& a) {
+    return a.f.mode == TTT_LN_RESIDUAL && (a.f.d == 16 || a.f.d == 32 || a.f.d == 64) && a.f.mini_batch >= 1 &&
+           a.f.mini_batch <= kMaxN;
+}
+
+size_t linear_backward_workspace_bytes(int B, int H, int T, int d, int mini_batch) {
+    if (B < 1 || H < 1 || T < 0 || d < 1 || mini_batch < 1) return 0;
+    const size_t nmb = ((size_t)T + mini_batch - 1) / mini_batch;
+    const size_t bh = (size_t)B * H;
+    return (bh * nmb * ((size_t)d * d + d) + bh * 2 * d) * sizeof(float);
+}
+
+cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cudaStream_t stream) {
+    if (!linear_backward_supports(a)) return cudaErrorInvalidValue;
+    const LinearArgs& f = a.f;
+    const int BH = f.B * f.H;
+    const size_t nmb = ((size_t)f.T + f.mini_batch - 1) / f.mini_batch;
+    float* states = workspace;
+    float* gb = workspace + (size_t)BH * nmb * ((size_t)f.d * f.d + f.d);
+    const size_t smem = sizeof(BwdSmem);
+    cudaError_t e;
+    if (f.dtype == TTT_BF16) {
+        auto* Q = static_cast<const __nv_bfloat16*>(f.Q);
+        auto* K = static_cast<const __nv_bfloat16*>(f.K);
+        auto* V = static_cast<const __nv_bfloat16*>(f.V);
+        if ((e = cudaFuncSetAttribute(ttt_linear_states_kernel<__nv_bfloat16>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(ttt_linear_backward_kernel<__nv_bfloat16>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        if (f.T > 0) {
+            ttt_linear_states_kernel<<<BH, kBwdThreads, smem, stream>>>(f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V,
+                                                                         f.eta, f.W0, f.b0, f.gamma, f.beta, f.H,
+                                                                         states);
+        }
+        ttt_linear_backward_kernel<<<BH, kBwdThreads, smem, stream>>>(
+            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T,
+            a.dQ, a.dK, a.dV, a.deta, a.dW0, a.db0, gb);
+    } else {
+        auto* Q = static_cast<const float*>(f.Q);
+        auto* K = static_cast<const float*>(f.K);
+        auto* V = static_cast<const float*>(f.V);
+        if ((e = cudaFuncSetAttribute(ttt_linear_states_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(ttt_linear_backward_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        if (f.T > 0) {
+            ttt_linear_states_kernel<<<BH, kBwdThreads, smem, stream>>>(f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V,
+                                                                         f.eta, f.W0, f.b0, f.gamma, f.beta, f.H,
+                                                                         states);
+        }
+        ttt_linear_backward_kernel<<<BH, kBwdThreads, smem, stream>>>(
+            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T,
+            a.dQ, a.dK, a.dV, a.deta, a.dW0, a.db0, gb);
+    }
+    const int hd = f.H * f.d;
+    ttt_linear_dgamma_kernel<<<(hd + 255) / 256, 256, 0, stream>>>(f.B, f.H, f.d, gb, a.dgamma, a.dbeta);
+    return cudaPeekAtLastError();
+}
+
+}  // namespace ttt

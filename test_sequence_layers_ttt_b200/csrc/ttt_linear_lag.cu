@@ -699,12 +699,15 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     }
 }
 
-int drop_chunk_from_env() {
-    const char* v = std::getenv("TTT_DEBUG_DROP_CHUNK");
-    return (v && v[0]) ? std::atoi(v) : -1;
-}
-
 }  // namespace
+
+int drop_chunk_hook() {
+    static const int c = [] {
+        const char* v = std::getenv("TTT_DEBUG_DROP_CHUNK");
+        return (v && v[0]) ? std::atoi(v) : -1;
+    }();
+    return c;
+}
 
 bool linear_tc_supports(const LinearArgs& a) {
     return a.d == D && a.dtype == TTT_BF16 && a.mode == TTT_LN_RESIDUAL && a.mini_batch == kChunk && a.T > 0 &&
@@ -722,7 +725,7 @@ cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(ttt_linear_lag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ttt_linear_lag_kernel<<<BH, kThreads, smem, stream>>>(mk, mv, mq, me, a.T, a.H, a.ln_eps, a.W0, a.b0, a.gamma,
-                                                           a.beta, a.Z, a.W_T, a.b_T, drop_chunk_from_env());
+                                                           a.beta, a.Z, a.W_T, a.b_T, drop_chunk_hook());
     return cudaPeekAtLastError();
 }
 

@@ -24,7 +24,7 @@ OK, NULL, SHAPE, DTYPE, ALIGN, ALIAS, UNSUP = 0, 1, 2, 3, 4, 5, 6
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:ttt_status|ttt_impl|const char\*|int)\s+(ttt_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:ttt_status|ttt_impl|const char\*|int|size_t)\s+(ttt_\w+)\s*\(",
                                  text, re.M)))
 
 
@@ -45,7 +45,7 @@ def test_status_strings():
     for code, name in enumerate(b.STATUS):
         assert b.status_string(code).startswith(name)
     assert b.status_string(99) == "TTT_ERR_UNKNOWN"
-    assert b.lib.ttt_abi_version() == 101
+    assert b.lib.ttt_abi_version() == 102
 
 
 # Fake, 16-byte aligned, non-overlapping device addresses.  Never dereferenced:
@@ -249,3 +249,52 @@ def test_empty_sequence_allows_null_token_buffers_but_not_state():
         p[i] = None
     p[4] = None  # W0 is still required
     assert linear_call(T=0, ptrs=p) == NULL
+
+
+# ---------------------------------------------------------------- layer backward (host validation only)
+# argument order: Q K V eta W0 b0 gamma beta dZ dW_T db_T dQ dK dV deta dW0 db0 dgamma dbeta workspace
+def backward_call(B=1, H=2, T=64, d=64, mb=16, dtype=0, mode=0, eps=1e-6, ptrs=None, ws_bytes=None):
+    p = [fake(i) for i in range(20)] if ptrs is None else ptrs
+    need = b.lib.ttt_linear_backward_workspace_size(B, H, T, d, mb)
+    ws = need if ws_bytes is None else ws_bytes
+    return b.lib.ttt_linear_backward(B, H, T, d, mb, dtype, mode, eps, *p, ctypes.c_size_t(ws), None)
+
+
+def test_backward_workspace_size_formula():
+    B, H, T, d, mb = 2, 3, 40, 64, 16
+    nmb = -(-T // mb)
+    assert b.linear_backward_workspace_size(B, H, T, d, mb) == 4 * (B * H * nmb * (d * d + d) + B * H * 2 * d)
+    assert b.linear_backward_workspace_size(0, 1, 1, 64, 16) == 0
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4, 5, 6, 7, 8, 11, 12, 13, 14, 15, 16, 17, 18, 19])
+def test_backward_null_required_pointer(idx):
+    p = [fake(k) for k in range(20)]
+    p[idx] = None
+    expected = b.STATUS.index("TTT_ERR_WORKSPACE") if idx == 19 else NULL
+    assert backward_call(ptrs=p) == expected
+
+
+def test_backward_state_gradients_may_be_null_and_workspace_is_checked():
+    p = [fake(k) for k in range(20)]
+    p[9] = p[10] = None
+    assert backward_call(ptrs=p, ws_bytes=16) == b.STATUS.index("TTT_ERR_WORKSPACE")
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=1), UNSUP), (dict(mb=32), UNSUP), (dict(d=48), UNSUP), (dict(mb=0), SHAPE), (dict(B=0), SHAPE),
+    (dict(dtype=4), DTYPE), (dict(eps=0.0), SHAPE)])
+def test_backward_bad_shapes(kw, code):
+    assert backward_call(**kw) == code
+
+
+def test_backward_alias_and_align():
+    p = [fake(k) for k in range(20)]
+    p[11] = p[8] + 256  # dQ inside dZ
+    assert backward_call(ptrs=p) == ALIAS
+    p = [fake(k) for k in range(20)]
+    p[15] = p[19] + 64  # dW0 inside the workspace
+    assert backward_call(ptrs=p) == ALIAS
+    p = [fake(k) for k in range(20)]
+    p[14] = fake(14) + 4
+    assert backward_call(ptrs=p) == ALIGN

@@ -1,0 +1,129 @@
+"""The TTT-Linear layer backward on the GPU (through the C ABI) against the
+float64 backward oracle (oracle/backward.py: torch autograd over a
+token-by-token restatement of the scan, pinned to the C oracle and to finite
+differences).  Both sides read identical input bits.
+
+Bar: every gradient within 1e-3 of its own RMS (max abs error).  The kernel
+runs in fp32; its error grows through the reverse sweep over the mini-batches
+and through the second-order LayerNorm terms, so the bar is looser than the
+forward's fp32 1e-4.  ("Learning to (Learn at Test Time)", literature record,
+Key takeaways bullet 2: the outer loop trains theta_K, theta_V, theta_Q, the
+initial weights and the learning rate.)
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import backward as ob
+from test_sequence_layers_ttt_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+BAR = 1e-3
+NAMES = ("dQ", "dK", "dV", "deta", "dW0", "db0", "dgamma", "dbeta")
+
+
+@pytest.fixture(scope="module")
+def ttt(cuda_device):
+    from test_sequence_layers_ttt_b200 import _binding
+    return _binding
+
+
+def rms(x):
+    return float(np.sqrt(np.mean(np.square(np.asarray(x, dtype=np.float64)))))
+
+
+def upstream(w, seed, with_state=True):
+    g = torch.Generator().manual_seed(1000 + seed)
+    dZ = torch.randn((w.B, w.H, w.T, w.d), generator=g)
+    dW = torch.randn((w.B, w.H, w.d, w.d), generator=g) if with_state else None
+    db = torch.randn((w.B, w.H, w.d), generator=g) if with_state else None
+    return dZ, dW, db
+
+
+def check(ttt, w, inp, dZ, dW, db, mb):
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    cu = lambda t: None if t is None else t.cuda()
+    got = ttt.ttt_linear_backward(*(cu(inp[k]) for k in keys), cu(dZ), cu(dW), cu(db), mini_batch=mb,
+                                  ln_eps=w.ln_eps)
+    torch.cuda.synchronize()
+    ref = ob.ttt_linear_backward(*(inp[k] for k in keys), dZ, mb, ln_eps=w.ln_eps,
+                                 dW_T=None if dW is None else dW, db_T=None if db is None else db)
+    worst = {}
+    for name, a, r in zip(NAMES, got, ref):
+        a = a.cpu().numpy().astype(np.float64)
+        assert np.isfinite(a).all(), f"{name}: non-finite"
+        err = float(np.abs(a - r).max()) / rms(r)
+        worst[name] = err
+        assert err <= BAR, f"{name}: max err {err:.2e} of RMS > {BAR}"
+    return worst
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+@pytest.mark.parametrize("name,shape,mb", [
+    ("linear_125m_2k", dict(B=1, H=2, T=48), 16),        # bf16, three mini-batches
+    ("linear_125m_2k", dict(B=2, H=3, T=40), 16),        # ragged last mini-batch
+    ("linear_125m_2k", dict(B=1, H=2, T=24), 8),
+    ("linear_125m_2k", dict(B=1, H=2, T=7), 1),           # online GD
+    ("linear_tiny_f32", {}, 16),                          # fp32, d = 16
+    ("linear_tiny_f32", dict(d=32, T=40), 4),
+])
+def test_linear_backward_vs_oracle(ttt, seed, name, shape, mb):
+    w = WORKLOADS[name].with_shape(**shape) if shape else WORKLOADS[name]
+    inp = make_inputs(w, seed)
+    check(ttt, w, inp, *upstream(w, seed), mb)
+
+
+def test_linear_backward_without_state_gradients(ttt):
+    """dW_T, db_T NULL: only the output's gradient flows back."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=64)
+    inp = make_inputs(w, 3)
+    check(ttt, w, inp, *upstream(w, 3, with_state=False), 16)
+
+
+def test_linear_backward_125m_heads(ttt):
+    """Every head of the 125M-layer shape (B = 8, H = 12, d = 64, b = 16, bf16
+    Q/K/V), on 256 tokens (the oracle's autograd loop bounds T)."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(T=256)
+    inp = make_inputs(w, 0)
+    check(ttt, w, inp, *upstream(w, 0), 16)
+
+
+def test_linear_backward_empty_sequence(ttt):
+    """T = 0: dW0 = dW_T, db0 = db_T, dgamma = dbeta = 0."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=0)
+    g = {k: v.cuda() for k, v in make_inputs(w, 1).items()}
+    dZ, dW, db = (None if t is None else t.cuda() for t in upstream(w, 1))
+    out = ttt.ttt_linear_backward(g["Q"], g["K"], g["V"], g["eta"], g["W0"], g["b0"], g["gamma"], g["beta"], dZ,
+                                  dW, db)
+    torch.cuda.synchronize()
+    assert torch.equal(out[4], dW) and torch.equal(out[5], db)
+    assert not out[6].any() and not out[7].any()
+
+
+def test_linear_backward_refuses_small_workspace_and_plain_mode(ttt):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=1, T=32)
+    g = {k: v.cuda() for k, v in make_inputs(w, 0).items()}
+    dZ = torch.zeros((1, 1, 32, 64), device="cuda")
+    args = (g["Q"], g["K"], g["V"], g["eta"], g["W0"], g["b0"], g["gamma"], g["beta"], dZ)
+    need = ttt.linear_backward_workspace_size(1, 1, 32, 64, 16)
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_linear_backward(*args, workspace=small)
+    assert ei.value.status == 9
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_linear_backward(*args, mode="plain")
+    assert ei.value.status == 6
+
+
+def test_linear_backward_is_deterministic(ttt):
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=3, H=2, T=64)
+    g = {k: v.cuda() for k, v in make_inputs(w, 4).items()}
+    dZ, dW, db = (t.cuda() for t in upstream(w, 4))
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    a = ttt.ttt_linear_backward(*(g[k] for k in keys), dZ, dW, db)
+    b = ttt.ttt_linear_backward(*(g[k] for k in keys), dZ, dW, db)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))

@@ -73,6 +73,19 @@ def test_reference_arm_under_torchrun_prints_once():
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
 
 
+def test_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` run without torchrun starts two ranks on this node
+    (the same line as under torchrun: rank 0 prints it once)."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", MASTER_PORT=str(_free_port()))
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--workload",
+           "linear_125m_2k", "--steps", "1", "--warmup", "0", "--ref-seconds", "0.2"]
+    p = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
 @pytest.mark.parametrize("world,ms", [(1, 2.0), (2, 2.0), (8, 4.0)])
 def test_weak_scaling_value_counts_every_rank(world, ms):
     sys.path.insert(0, ROOT)

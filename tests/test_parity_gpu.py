@@ -69,7 +69,7 @@ def compare_linear(ttt, w, inp, impl="auto", mini_batch=None):
     e = assert_close(Z, Zo, f, "Z")
     assert_close(W_T, Wo, f, "W_T")
     if b_T is not None and np.any(bo):
-        assert_close(b_T, bo, f, "b_T", denom=max(rms(bo), rms(Wo)))
+        assert_close(b_T, bo, f, "b_T")
     return e
 
 
@@ -105,62 +105,120 @@ def test_linear_bf16_reduced(ttt, seed, name, shape, impl):
     compare_linear(ttt, w, make_inputs(w, seed), impl)
 
 
-@pytest.mark.parametrize("impl", ["auto", "tensorcore"])
+# the tensor-core families of TTT-Linear: warp-level mma with the state in
+# registers, and the state products on tcgen05 with TMEM accumulators
+TC_LINEAR = ["tensorcore", "tcgen05"]
+
+
+@pytest.mark.parametrize("impl", ["auto"] + TC_LINEAR)
 def test_linear_125m_full(ttt, impl):
     w = WORKLOADS["linear_125m_2k"]
     compare_linear(ttt, w, make_inputs(w, 0), impl)
 
 
+@pytest.mark.parametrize("impl", TC_LINEAR)
 @pytest.mark.parametrize("seed", [0, 1, 2])
-@pytest.mark.parametrize("shape", [dict(B=1, H=1, T=16), dict(B=1, H=2, T=48), dict(B=2, H=3, T=256),
-                                   dict(B=1, H=4, T=1024)])
-def test_linear_tensorcore_shapes(ttt, seed, shape):
-    """The tensor-core family on 1, 3, 16 and 64 chunks (the 8-stage ring wraps)."""
+@pytest.mark.parametrize("shape", [dict(B=1, H=1, T=16), dict(B=1, H=1, T=32), dict(B=1, H=2, T=48),
+                                   dict(B=2, H=3, T=256), dict(B=1, H=4, T=1024)])
+def test_linear_tensorcore_shapes(ttt, seed, shape, impl):
+    """The tensor-core families on 1, 2, 3, 16 and 64 chunks (every ring wraps)."""
     w = WORKLOADS["linear_1p3b_32k"].with_shape(**shape)
-    compare_linear(ttt, w, make_inputs(w, seed), "tensorcore")
+    compare_linear(ttt, w, make_inputs(w, seed), impl)
 
 
-def test_linear_tensorcore_matches_generic_closely(ttt):
-    """Both CUDA families agree far inside the oracle tolerance."""
+@pytest.mark.parametrize("impl", TC_LINEAR)
+def test_linear_tensorcore_matches_generic_closely(ttt, impl):
+    """The CUDA families agree far inside the oracle tolerance."""
     w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=2, T=512)
     inp = make_inputs(w, 9)
-    Zt, Wt_, _ = gpu_linear(ttt, w, inp, "tensorcore")
+    Zt, Wt_, _ = gpu_linear(ttt, w, inp, impl)
     Zg, Wg, _ = gpu_linear(ttt, w, inp, "generic")
-    assert_close(Zt, Zg, 1e-3, "Z tensorcore vs generic")
+    assert_close(Zt, Zg, 1e-3, f"Z {impl} vs generic")
+    assert_close(Wt_, Wg, 1e-3, f"W_T {impl} vs generic")
 
 
-def test_linear_bounded_wait_times_out_and_context_survives(ttt, monkeypatch):
-    """Fault injection on the host side of a bounded wait: the producer is told
+@pytest.mark.parametrize("impl", TC_LINEAR + ["generic"])
+@pytest.mark.parametrize("offset", [4.0, -2.5])
+def test_linear_bias_with_large_mean(ttt, impl, offset):
+    """b0 with a mean far above the spread of x W (b0 = offset + N(0, 0.02^2)):
+    the mean of y = x W + b is then large against its spread, where a one-pass
+    variance in fp32 would cancel; W0 gets a row-mean offset as well."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=2, T=512)
+    inp = make_inputs(w, 11)
+    gen = torch.Generator().manual_seed(123)
+    inp["b0"] = (offset + 0.02 * torch.randn(inp["b0"].shape, generator=gen)).float()
+    inp["W0"] = (inp["W0"] + 0.3 * torch.randn(inp["W0"].shape[:-1] + (1,), generator=gen)).float()
+    compare_linear(ttt, w, inp, impl)
+
+
+_FAULT_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[2])
+import oracle
+from test_sequence_layers_ttt_b200 import _binding as ttt
+from test_sequence_layers_ttt_b200.inputs import WORKLOADS, make_inputs
+keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+impl = sys.argv[1]
+w = WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=2, T=256)
+g = {k: v.cuda() for k, v in make_inputs(w, 0).items()}
+try:
+    ttt.ttt_linear_forward(*(g[k] for k in keys), impl=impl)
+    print("NO_TIMEOUT")
+except ttt.TTTError as e:
+    print("STATUS", e.status)
+torch.cuda.synchronize()
+# the same context, a sequence of three chunks (chunk 3 does not exist, so the hook never fires)
+w3 = w.with_shape(T=48)
+inp = make_inputs(w3, 1)
+Z, W_T, b_T = ttt.ttt_linear_forward(*(inp[k].cuda() for k in keys), impl=impl)
+torch.cuda.synchronize()
+Zo, Wo, bo = oracle.ttt_linear(*(inp[k] for k in keys), 16)
+err = float(np.abs(Z.cpu().numpy() - Zo).max()) / float(np.sqrt(np.mean(Zo ** 2)))
+print("AFTER", err)
+"""
+
+
+@pytest.mark.parametrize("impl", TC_LINEAR)
+def test_linear_bounded_wait_times_out_and_context_survives(ttt, impl, tmp_path):
+    """Fault injection on the host side of a bounded wait, in a child process
+    (the library reads its environment once per process): the producer is told
     never to load chunk 3, so the consumers' wait for it runs out (about a
-    second), the kernel drains and returns, and TTT_CHECK=1 reports
-    TTT_ERR_TIMEOUT.  The next call on the same context is correct."""
-    w = WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=2, T=256)
-    inp = make_inputs(w, 0)
-    g = to_cuda(inp)
-    monkeypatch.setenv("TTT_CHECK", "1")
-    monkeypatch.setenv("TTT_DEBUG_DROP_CHUNK", "3")
-    with pytest.raises(ttt.TTTError) as ei:
-        ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl="tensorcore")
-    assert ei.value.status == 8
-    monkeypatch.delenv("TTT_DEBUG_DROP_CHUNK")
-    torch.cuda.synchronize()
-    compare_linear(ttt, w, inp, "tensorcore")
+    second), the kernel drains its loads and tensor-core work and returns, and
+    the call reports TTT_ERR_TIMEOUT.  A later call on the same context is
+    correct."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, TTT_CHECK="1", TTT_DEBUG_DROP_CHUNK="3")
+    r = subprocess.run([sys.executable, "-c", _FAULT_CHILD, impl, root], env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = r.stdout.split("\n")
+    assert "STATUS 8" in lines, r.stdout
+    after = [float(l.split()[1]) for l in lines if l.startswith("AFTER")]
+    assert after and after[0] <= TOL["bf16"], r.stdout
 
 
-def test_linear_1p3b_32k_full_sampled_heads(ttt):
-    """The benchmarked launch: all 64 scans of 32k tokens on the GPU, four of
-    them checked end to end against the oracle."""
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_linear_1p3b_32k_full_all_scans(ttt, seed):
+    """The benchmarked launch: all 64 scans of 32k tokens on the GPU, every one
+    checked end to end against the oracle."""
     w = WORKLOADS["linear_1p3b_32k"]
-    inp = make_inputs(w, 0)
+    inp = make_inputs(w, seed)
     Z, W_T, b_T = gpu_linear(ttt, w, inp)
-    pairs = [(0, 0), (0, 17), (1, 5), (1, 31)]
-    sel = select_heads(inp, pairs)
-    Zo, Wo, bo = oracle_linear(w, sel)
+    Zo, Wo, bo = oracle_linear(w, inp)
     f = TOL["bf16"]
-    for i, (bb, hh) in enumerate(pairs):
-        assert_close(Z[bb, hh], Zo[0, i], f, f"Z[{bb},{hh}]", denom=rms(Zo))
-        assert_close(W_T[bb, hh], Wo[0, i], f, f"W_T[{bb},{hh}]", denom=rms(Wo))
-    assert np.isfinite(Z).all()
+    assert_close(Z, Zo, f, "Z")
+    assert_close(W_T, Wo, f, "W_T")
+    assert_close(b_T, bo, f, "b_T")
+
+
+@pytest.mark.parametrize("impl", TC_LINEAR)
+def test_linear_1p3b_32k_full_each_tensorcore_family(ttt, impl):
+    """Each tensor-core family on the full 1.3B/32k launch, all 64 scans."""
+    w = WORKLOADS["linear_1p3b_32k"]
+    compare_linear(ttt, w, make_inputs(w, 1), impl)
 
 
 @pytest.mark.parametrize("mb", [1, 2, 4, 8, 32, 64])
@@ -190,7 +248,7 @@ def test_linear_short_and_empty_sequences(ttt, T):
         compare_linear(ttt, w, inp)
 
 
-@pytest.mark.parametrize("impl", ["generic", "tensorcore"])
+@pytest.mark.parametrize("impl", ["generic"] + TC_LINEAR)
 def test_linear_in_place_state_and_continuation(ttt, impl):
     """W_T may be W0 (in-place).  Splitting the sequence at a mini-batch
     boundary and feeding the state back continues the same computation:
@@ -216,7 +274,7 @@ def test_linear_in_place_state_and_continuation(ttt, impl):
         assert_close(W.cpu().numpy(), Wf.cpu().numpy(), 1e-4, "W continuation")
 
 
-@pytest.mark.parametrize("impl", ["auto", "generic", "tensorcore"])
+@pytest.mark.parametrize("impl", ["auto", "generic"] + TC_LINEAR)
 def test_linear_deterministic(ttt, impl):
     w = WORKLOADS["linear_1p3b_32k"].with_shape(B=2, H=4, T=512)
     g = to_cuda(make_inputs(w, 7))
@@ -226,11 +284,12 @@ def test_linear_deterministic(ttt, impl):
     assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
-def test_linear_tensorcore_refuses_other_shapes(ttt):
+@pytest.mark.parametrize("impl", TC_LINEAR)
+def test_linear_tensorcore_refuses_other_shapes(ttt, impl):
     w = WORKLOADS["linear_tiny_f32"]
     g = to_cuda(make_inputs(w, 0))
     with pytest.raises(ttt.TTTError) as ei:
-        ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl="tensorcore")
+        ttt.ttt_linear_forward(*(g[k] for k in LINEAR_KEYS), impl=impl)
     assert ei.value.status == 6
 
 
@@ -310,7 +369,7 @@ def compare_decode(out, ref, f, plain):
         assert_close(out[i], ref[i], f, name)
     if not plain:
         for name, i in (("b", 2), ("b_mb", 4)):
-            assert_close(out[i], ref[i], f, name, denom=max(rms(ref[i]), rms(ref[1])))
+            assert_close(out[i], ref[i], f, name)
 
 
 @pytest.mark.parametrize("name,shape,mb,cuts", [
@@ -341,7 +400,7 @@ def test_linear_decode_token_by_token_equals_forward_oracle(ttt):
     f = TOL[w.dtype]
     assert_close(out[0], Zo, f, "Z")
     assert_close(out[1], Wo, f, "W")
-    assert_close(out[2], bo, f, "b", denom=max(rms(bo), rms(Wo)))
+    assert_close(out[2], bo, f, "b")
 
 
 def test_linear_decode_one_call_is_the_generic_forward(ttt):
@@ -552,12 +611,21 @@ def test_mlp_f32_inputs(ttt):
     compare_mlp(ttt, w, make_inputs(w, 2))
 
 
-def test_mlp_full_sampled_heads(ttt):
-    """The benchmarked launch (the split tensor-core family): all 48 scans of 8k
-    tokens on the GPU, three checked end to end against the oracle."""
+def test_mlp_auto_picks_split_on_the_8k_workload(ttt):
+    """AUTO runs the split tensor-core family on the benchmarked 8k workload."""
     w = WORKLOADS["mlp_8k"]
     assert ttt.mlp_pick_impl(w.B, w.H, w.T, w.d, w.hidden, w.mini_batch, w.dtype) == "tensorcore_split"
-    compare_mlp(ttt, w, make_inputs(w, 0), pairs=[(0, 0), (2, 7), (3, 11)])
+
+
+@pytest.mark.parametrize("impl", TC_MLP)
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_mlp_full_all_scans(ttt, impl, seed):
+    """The full 8k TTT-MLP workload, all 48 scans checked against the oracle, for
+    each tensor-core family (seed 0 for the one-CTA family)."""
+    if impl == "tensorcore" and seed > 0:
+        pytest.skip("the one-CTA family is checked in full on one seed")
+    w = WORKLOADS["mlp_8k"]
+    compare_mlp(ttt, w, make_inputs(w, seed), impl=impl)
 
 
 @pytest.mark.parametrize("impl", TC_MLP)
@@ -567,13 +635,6 @@ def test_mlp_tensorcore_vs_oracle(ttt, T, seed, impl):
     """Several chunks, all heads of a small batch, each tensor-core family explicitly."""
     w = WORKLOADS["mlp_8k"].with_shape(B=2, H=3, T=T)
     compare_mlp(ttt, w, make_inputs(w, seed), impl=impl)
-
-
-def test_mlp_full_sampled_heads_one_cta_family(ttt):
-    """The one-CTA family on the full 8k workload, as AUTO runs it when 2 B H
-    CTAs no longer fit in one wave."""
-    w = WORKLOADS["mlp_8k"]
-    compare_mlp(ttt, w, make_inputs(w, 1), pairs=[(1, 3), (3, 0)], impl="tensorcore")
 
 
 def test_mlp_split_matches_one_cta_family(ttt):
