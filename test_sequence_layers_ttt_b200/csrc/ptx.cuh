@@ -159,5 +159,27 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
     lo = pack_hi_halves(__float_as_uint(x0 - __uint_as_float(h0)), __float_as_uint(x1 - __uint_as_float(h1)));
 }
 
+// Cheaper split for operands that are re-split every chunk: hi = x truncated to
+// bf16 (the top half of its bit pattern), lo = (x - hi) truncated to bf16; x - hi
+// is exact in fp32, so |x - hi - lo| < 2^-15 |x|.  Five instructions per pair:
+// two byte permutes, two masks and one packed fp32 subtraction.
+__device__ __forceinline__ void split_pair_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+    hi = __byte_perm(b0, b1, 0x7632);
+    const uint32_t t0 = b0 & 0xffff0000u, t1 = b1 & 0xffff0000u;
+    uint64_t d;
+    asm("{\n .reg .b64 a, b;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %4};\n sub.rn.f32x2 %0, a, b;\n}\n"
+        : "=l"(d) : "r"(b0), "r"(b1), "r"(t0), "r"(t1));
+    lo = __byte_perm((uint32_t)d, (uint32_t)(d >> 32), 0x7632);
+}
+// (x0, x1) += (y0, y1) as one packed fp32 add
+__device__ __forceinline__ void add2(float& x0, float& x1, float y0, float y1) {
+    uint64_t d;
+    asm("{\n .reg .b64 a, b;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %4};\n add.rn.f32x2 %0, a, b;\n}\n"
+        : "=l"(d) : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+    x0 = __uint_as_float((uint32_t)d);
+    x1 = __uint_as_float((uint32_t)(d >> 32));
+}
+
 }  // namespace ptx
 }  // namespace ttt

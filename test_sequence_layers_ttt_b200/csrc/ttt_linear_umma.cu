@@ -37,8 +37,9 @@
 //   PR  13    TMA loads of K, V, Q tiles (128-byte swizzle) and eta.
 //   PA  14    gamma * (x + beta - v) per (feature, token) and its row sums.
 //   PB  15    S1 (as mma B fragments), S2 and L (as hi/lo operand tiles).
-// Precision: every product with an fp32 operand splits it into bf16 hi + lo and
-// drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
+// Precision: every product with an fp32 operand splits it into bf16 hi + lo
+// (hi the truncated top half, lo the truncated remainder: |x - hi - lo| below
+// 2^-15 |x|) and drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
 // and added to the fp32 registers with fp32 adds (tensor-core accumulation of
 // thousands of increments would not round to nearest).
 // Feature order: accumulator row r = 16 j + i holds output feature
@@ -79,7 +80,10 @@ constexpr int TILE = kChunk * D * 2;  // one [16][64] bf16 tile
 constexpr uint32_t kStageTx = 3 * TILE + kChunk * 4;
 constexpr long long kTimeoutCycles = 2000000000LL;
 // TMEM columns
-constexpr uint32_t kColDW = 0, kColDB = 64, kColR = 128, kColZ = 192, kTmemCols = 256;
+constexpr uint32_t kColDW = 0, kColDB = 64, kColR = 128, kColZ = 192, kTmemCols = 512;
+// A operands in TMEM (the kAInTmem variant): W~^T hi (32 columns of bf16 pairs), lo (32), the bias
+// K step (8: column 0 holds b hi, b lo), and E_c hi (8), lo (8) per buffer
+constexpr uint32_t kColWA = 256, kColWB = 320, kColEA = 384;
 
 struct alignas(1024) Stage {
     unsigned char K[TILE], V[TILE], Q[TILE];
@@ -103,7 +107,7 @@ struct UmmaSmem {
     unsigned char ones16[16 * 32];         // [t][k]: k = 0, 1 are 1
     unsigned char ones8[8 * 32 + 128];     // [n][k]: row 0 is 1 for every k < 16
     PreSlot pre[NPRE];
-    alignas(16) float eta[NS][kChunk];
+    alignas(128) float eta[NS][32];         // TMA destinations: 128-byte aligned rows (16 used)
     float red_ch[2][kChunk][5][4];         // [buf][token][sum][warp]
     float coef_ch[4][kChunk][8];           // [warp][token][mu, a, b2, c2, d2]
     float red_ow[2][kChunk][2][4];
@@ -149,6 +153,7 @@ __device__ __forceinline__ void arrive1(uint64_t* bar, int lane) {
     if (lane == 0) ptx::mbar_arrive(bar);
 }
 
+template <bool kAInTmem>
 __global__ void __launch_bounds__(kThreads, 1)
 ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmEta,
@@ -381,18 +386,34 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 #pragma unroll
                 for (int ks = 0; ks < 4; ks++) {
                     const uint64_t b = tc05::desc_k128(tile, ks);
-                    tc05::mma_bf16_ss(tmem + dcol, tc05::desc_k128(whi, ks), b, I16, ks > 0);
-                    tc05::mma_bf16_ss(tmem + dcol, tc05::desc_k128(wlo, ks), b, I16, 1);
+                    if constexpr (kAInTmem) {
+                        tc05::mma_bf16_ts(tmem + dcol, tmem + kColWA + 8 * ks, b, I16, ks > 0);
+                        tc05::mma_bf16_ts(tmem + dcol, tmem + kColWA + 32 + 8 * ks, b, I16, 1);
+                    } else {
+                        tc05::mma_bf16_ss(tmem + dcol, tc05::desc_k128(whi, ks), b, I16, ks > 0);
+                        tc05::mma_bf16_ss(tmem + dcol, tc05::desc_k128(wlo, ks), b, I16, 1);
+                    }
                 }
-                tc05::mma_bf16_ss(tmem + dcol, d_bias, d_one16, I16, 1);
+                if constexpr (kAInTmem)
+                    tc05::mma_bf16_ts(tmem + dcol, tmem + kColWB, d_one16, I16, 1);
+                else
+                    tc05::mma_bf16_ss(tmem + dcol, d_bias, d_one16, I16, 1);
             };
-            // D += E^T M^T for a [16][16] hi/lo operand pair (hi*hi + hi*lo + lo*hi)
-            auto issue_corr = [&](uint32_t dcol, uint32_t ehi, uint32_t elo, uint32_t mhi, uint32_t mlo) {
-                const uint64_t eh = tc05::desc_k16(ehi), el = tc05::desc_k16(elo);
+            // D += E^T M^T for a [16][16] hi/lo operand pair (hi*hi + hi*lo + lo*hi); E buffer e
+            auto issue_corr = [&](uint32_t dcol, int e, uint32_t mhi, uint32_t mlo) {
                 const uint64_t mh = tc05::desc_k16(mhi), ml = tc05::desc_k16(mlo);
-                tc05::mma_bf16_ss(tmem + dcol, eh, mh, I16, 1);
-                tc05::mma_bf16_ss(tmem + dcol, eh, ml, I16, 1);
-                tc05::mma_bf16_ss(tmem + dcol, el, mh, I16, 1);
+                if constexpr (kAInTmem) {
+                    const uint32_t ea = tmem + kColEA + 16 * e;
+                    tc05::mma_bf16_ts(tmem + dcol, ea, mh, I16, 1);
+                    tc05::mma_bf16_ts(tmem + dcol, ea, ml, I16, 1);
+                    tc05::mma_bf16_ts(tmem + dcol, ea + 8, mh, I16, 1);
+                } else {
+                    const uint64_t eh = tc05::desc_k16(ptx::smem_addr(s.E[e][0]));
+                    const uint64_t el = tc05::desc_k16(ptx::smem_addr(s.E[e][1]));
+                    tc05::mma_bf16_ss(tmem + dcol, eh, mh, I16, 1);
+                    tc05::mma_bf16_ss(tmem + dcol, eh, ml, I16, 1);
+                    tc05::mma_bf16_ss(tmem + dcol, el, mh, I16, 1);
+                }
             };
             // prologue: W~_0 ready; R_0, R_1, R_2 = X~_j W~_0 (R_0, R_1 final), zbar_0 = Q~_0 W~_0
             ok = wait_k(&s.w_full, 0, abort_flag);
@@ -411,13 +432,22 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 if (ok && c >= 2) ok = wait_k(&s.dw_empty, c - 2, abort_flag);
                 if (!ok) break;
                 tc05::fence_after_sync();
-                const uint32_t ehi = ptx::smem_addr(s.E[e][0]), elo = ptx::smem_addr(s.E[e][1]);
                 {
                     const uint64_t xmn = tc05::desc_mn128(ptx::smem_addr(s.st[(c - 1) % NS].K));
-                    tc05::mma_bf16_ss(tmem + kColDW, tc05::desc_k16(ehi), xmn, I64, 0);
-                    tc05::mma_bf16_ss(tmem + kColDW, tc05::desc_k16(elo), xmn, I64, 1);
-                    tc05::mma_bf16_ss(tmem + kColDB, tc05::desc_k16(ehi), d_one8, I8, 0);
-                    tc05::mma_bf16_ss(tmem + kColDB, tc05::desc_k16(elo), d_one8, I8, 1);
+                    if constexpr (kAInTmem) {
+                        const uint32_t ea = tmem + kColEA + 16 * e;
+                        tc05::mma_bf16_ts(tmem + kColDW, ea, xmn, I64, 0);
+                        tc05::mma_bf16_ts(tmem + kColDW, ea + 8, xmn, I64, 1);
+                        tc05::mma_bf16_ts(tmem + kColDB, ea, d_one8, I8, 0);
+                        tc05::mma_bf16_ts(tmem + kColDB, ea + 8, d_one8, I8, 1);
+                    } else {
+                        const uint64_t eh = tc05::desc_k16(ptx::smem_addr(s.E[e][0]));
+                        const uint64_t el = tc05::desc_k16(ptx::smem_addr(s.E[e][1]));
+                        tc05::mma_bf16_ss(tmem + kColDW, eh, xmn, I64, 0);
+                        tc05::mma_bf16_ss(tmem + kColDW, el, xmn, I64, 1);
+                        tc05::mma_bf16_ss(tmem + kColDB, eh, d_one8, I8, 0);
+                        tc05::mma_bf16_ss(tmem + kColDB, el, d_one8, I8, 1);
+                    }
                 }
                 tc05::commit(ptx::smem_addr(&s.dw_full));
                 tc05::commit(ptx::smem_addr(&s.in_empty[(c - 1) % NS]));
@@ -426,14 +456,14 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                     const int p1 = (c + 1) % NPRE;
                     ok = wait_k(&s.pre_full[p1], (c + 1) / NPRE, abort_flag);
                     if (!ok) break;
-                    issue_corr(kColR + 16 * ((c + 1) % NR), ehi, elo, ptx::smem_addr(s.pre[p1].s2[0]),
+                    issue_corr(kColR + 16 * ((c + 1) % NR), e, ptx::smem_addr(s.pre[p1].s2[0]),
                                ptx::smem_addr(s.pre[p1].s2[1]));
                     tc05::commit(ptx::smem_addr(&s.r_full[(c + 1) % NR]));
                 }
                 // ---- zbar_{c-1} += E_{c-1}^T L_{c-1}^T
                 ok = wait_k(&s.pre_full[pc], (c - 1) / NPRE, abort_flag);
                 if (!ok) break;
-                issue_corr(kColZ + 16 * ((c - 1) % NZ), ehi, elo, ptx::smem_addr(s.pre[pc].l[0]),
+                issue_corr(kColZ + 16 * ((c - 1) % NZ), e, ptx::smem_addr(s.pre[pc].l[0]),
                            ptx::smem_addr(s.pre[pc].l[1]));
                 tc05::commit(ptx::smem_addr(&s.z_full[(c - 1) % NZ]));
                 tc05::commit(ptx::smem_addr(&s.e_empty[e]));
@@ -503,7 +533,30 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             bt0 = b0[(size_t)bh * D + f0] - s.u[D];
             bt1 = b0[(size_t)bh * D + f1] - s.u[D];
         }
+        const uint32_t tq = tmem + tc05::taddr_lane(32 * q);
+        if constexpr (kAInTmem) tc05::st_16x128b_x2(tq + kColWB, 0u, 0u, 0u, 0u);  // bias K step: zeros
         auto write_tiles = [&]() {
+            if constexpr (kAInTmem) {
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    ptx::split_pair_trunc(Wt[4 * j + 0], Wt[4 * j + 1], hi[2 * j], lo[2 * j]);
+                    ptx::split_pair_trunc(Wt[4 * j + 2], Wt[4 * j + 3], hi[2 * j + 1], lo[2 * j + 1]);
+                }
+                tc05::st_16x128b_x8(tq + kColWA, hi);
+                tc05::st_16x128b_x8(tq + kColWA + 32, lo);
+                uint32_t bb0 = 0u, bb1 = 0u;  // bias row: k = 0 holds b hi, k = 1 holds b lo
+                if (t4 == 0) {
+                    uint32_t h, l;
+                    ptx::split_pair(bt0, 0.f, h, l);
+                    bb0 = (h & 0xffffu) | (l << 16);
+                    ptx::split_pair(bt1, 0.f, h, l);
+                    bb1 = (h & 0xffffu) | (l << 16);
+                }
+                tc05::st_16x128b_x1(tq + kColWB, bb0, bb1);
+                tc05::wait_st();
+                tc05::fence_before_sync();
+            } else {
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 uint32_t h0, l0, h1, l1;
@@ -523,10 +576,10 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 *reinterpret_cast<uint32_t*>(s.Abias + tc05::kmajor16_offset(r1, 0)) = (h & 0xffffu) | (l << 16);
             }
             ptx::fence_proxy_async_smem();
+            }
             arrive1(&s.w_full, lane);
         };
         write_tiles();  // W~_0
-        const uint32_t tq = tmem + tc05::taddr_lane(32 * q);
         for (int c = 0; c < n; c++) {
             wait_k(&s.dw_full, c, abort_flag);
             tc05::fence_after_sync();
@@ -537,7 +590,7 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             tc05::fence_before_sync();
             arrive1(&s.dw_empty, lane);
 #pragma unroll
-            for (int i = 0; i < 32; i++) Wt[i] += dv[i];
+            for (int i = 0; i < 32; i += 2) ptx::add2(Wt[i], Wt[i + 1], dv[i], dv[i + 1]);
             if (t4 == 0) {
                 bt0 += db[0];
                 bt1 += db[2];
@@ -700,13 +753,20 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                     E[nt][2 + e] = fmaf(cf.y, gc[4 * nt + 2 + e], fmaf(fmaf(cf.z, ga1, cf.w), m1, d2));
                 }
             // E_c as A fragments (rows r0/r1, k = tokens) and as hi/lo operand tiles
-            ptx::split_pair(E[0][0], E[0][1], ah[0], al[0]);
-            ptx::split_pair(E[0][2], E[0][3], ah[1], al[1]);
-            ptx::split_pair(E[1][0], E[1][1], ah[2], al[2]);
-            ptx::split_pair(E[1][2], E[1][3], ah[3], al[3]);
+            ptx::split_pair_trunc(E[0][0], E[0][1], ah[0], al[0]);
+            ptx::split_pair_trunc(E[0][2], E[0][3], ah[1], al[1]);
+            ptx::split_pair_trunc(E[1][0], E[1][1], ah[2], al[2]);
+            ptx::split_pair_trunc(E[1][2], E[1][3], ah[3], al[3]);
             const int eb = c % NE;
             if (c >= NE) wait_k(&s.e_empty[eb], c / NE - 1, abort_flag);
-            {
+            if constexpr (kAInTmem) {
+                tc05::fence_after_sync();
+                const uint32_t ea = tq + kColEA + 16 * eb;
+                tc05::st_16x128b_x2(ea, ah[0], ah[1], ah[2], ah[3]);
+                tc05::st_16x128b_x2(ea + 8, al[0], al[1], al[2], al[3]);
+                tc05::wait_st();
+                tc05::fence_before_sync();
+            } else {
                 unsigned char* th = s.E[eb][0];
                 unsigned char* tl = s.E[eb][1];
                 const uint32_t o00 = tc05::kmajor16_offset(r0, 2 * t4), o10 = tc05::kmajor16_offset(r0 + 8, 2 * t4);
@@ -720,7 +780,7 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 *reinterpret_cast<uint32_t*>(tl + o01) = al[2];
                 *reinterpret_cast<uint32_t*>(tl + o11) = al[3];
             }
-            ptx::fence_proxy_async_smem();
+            if constexpr (!kAInTmem) ptx::fence_proxy_async_smem();
             arrive1(&s.e_full[eb], lane);
             if (c + 1 < n) load_inputs(c + 1);
         }
@@ -809,6 +869,14 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 
 }  // namespace
 
+// Where the MMAs read their A operands (the state and E_c): tensor memory, written by the warps that
+// hold them with tcgen05.st, or shared-memory tiles.
+#ifndef TTT_UMMA_A_IN_SMEM
+constexpr bool kUmmaAInTmem = true;
+#else
+constexpr bool kUmmaAInTmem = false;
+#endif
+
 bool linear_umma_supports(const LinearArgs& a) {
     return a.d == D && a.dtype == TTT_BF16 && a.mode == TTT_LN_RESIDUAL && a.mini_batch == kChunk && a.T > 0 &&
            a.T % kChunk == 0;
@@ -822,10 +890,11 @@ cudaError_t launch_linear_umma(const LinearArgs& a, cudaStream_t stream) {
         !make_token_tile_map(&mq, a.Q, a.T, BH) || !make_eta_row_map(&me, a.eta, a.T, BH))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(UmmaSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(ttt_linear_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kernel = kUmmaAInTmem ? ttt_linear_umma_kernel<true> : ttt_linear_umma_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    ttt_linear_umma_kernel<<<BH, kThreads, smem, stream>>>(mk, mv, mq, me, a.T, a.H, a.ln_eps, a.W0, a.b0, a.gamma,
-                                                            a.beta, a.Z, a.W_T, a.b_T, drop_chunk_hook());
+    kernel<<<BH, kThreads, smem, stream>>>(mk, mv, mq, me, a.T, a.H, a.ln_eps, a.W0, a.b0, a.gamma, a.beta, a.Z,
+                                           a.W_T, a.b_T, drop_chunk_hook());
     return cudaPeekAtLastError();
 }
 
