@@ -112,11 +112,16 @@ typedef enum {
     TTT_IMPL_TENSORCORE_SPLIT = 3, /* TTT-MLP only, same shapes as TTT_IMPL_TENSORCORE: each
                                       scan's hidden units split over the two CTAs of a
                                       cluster (two SMs per scan) */
-    TTT_IMPL_TCGEN05 = 4 /* TTT-Linear only, same shapes as TTT_IMPL_TENSORCORE: the products
+    TTT_IMPL_TCGEN05 = 4, /* TTT-Linear only, same shapes as TTT_IMPL_TENSORCORE: the products
                             with the state run on the 5th-generation tensor cores (tcgen05,
                             fp32 accumulators in tensor memory, one issuing thread), the
                             sequential per-chunk chain on warp-level mma; the state is kept
                             centred on its per-row means, which are added back to W_T, b_T */
+    TTT_IMPL_TENSORCORE_LAG2 = 5 /* TTT-Linear only, same shapes as TTT_IMPL_TENSORCORE: the state
+                                    increment on tcgen05 (fp32 in tensor memory), the products with
+                                    the state and the per-chunk chain on warp-level mma, with two
+                                    chunks of slack between the state and the chain; the state is
+                                    kept centred as in TTT_IMPL_TCGEN05 */
 } ttt_impl;
 
 /*
@@ -244,6 +249,35 @@ ttt_status ttt_mlp_decode_impl(int B, int H, int T, int d, int hidden, int mini_
  * TTT_IMPL_TENSORCORE. */
 ttt_impl ttt_mlp_pick_impl(int B, int H, int T, int d, int hidden, int mini_batch,
                            ttt_dtype qkv_dtype);
+
+/*
+ * The layer's prologue: the scan's inputs from the layer input x, in one kernel
+ * (literature record, Key takeaways bullets 1 and 2: the scan sees the views
+ * theta_K x_t, theta_V x_t, theta_Q x_t of each token and a learning rate that
+ * depends on the token; the codewithpapers.app record names the official
+ * code's rotate_half helper).  Per head h and token t (readings of the pages,
+ * which give no formulas):
+ *   Q = x theta_q[h], K = x theta_k[h], V = x theta_v[h]        (no bias)
+ *   eta = eta_base * sigmoid(x . theta_lr[h] + b_lr[h]) / d
+ *   rotary (when rotary != 0), on Q and K: features i and i + d/2 rotate
+ *   together by the angle p * rope_base^(-2 i / d), p = pos0 + t the token's
+ *   absolute position.
+ *   x         [B][T][d_model] bf16
+ *   theta_q, theta_k, theta_v  [H][d_model][d] bf16;  theta_lr [H][d_model] bf16
+ *   b_lr      [H] fp32
+ *   Q, K, V   [B][H][T][d] bf16 outputs (the layout ttt_linear_forward reads),
+ *             rounded to nearest from the fp32 accumulation
+ *   eta       [B][H][T] fp32 output
+ * Built for d = 64, d_model a multiple of 64, H a multiple of 4 up to 256
+ * (TTT_ERR_UNSUPPORTED otherwise); T >= 1.  Runs on the tcgen05 tensor cores
+ * (bf16 products, fp32 accumulation).  Outputs may not overlap the inputs or
+ * each other (TTT_ERR_ALIAS).  Other conventions as ttt_linear_forward.
+ */
+ttt_status ttt_prologue_forward(int B, int T, int H, int d, int d_model, int pos0, float eta_base,
+                                float rope_base, int rotary, const void* x, const void* theta_q,
+                                const void* theta_k, const void* theta_v, const void* theta_lr,
+                                const float* b_lr, void* Q, void* K, void* V, float* eta,
+                                ttt_stream_t stream);
 
 /*
  * TTT-Linear layer backward: the gradients an outer training loop needs

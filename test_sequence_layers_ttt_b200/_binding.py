@@ -19,12 +19,14 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
+# TTT_B200_LIBRARY may name another build of the same library (the timeline build)
+LIB_PATH = os.environ.get("TTT_B200_LIBRARY") or os.path.join(_PKG, "libttt_b200.so")
 
 TTT_BF16, TTT_F32 = 0, 1
 TTT_LN_RESIDUAL, TTT_PLAIN = 0, 1
-IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3, "tcgen05": 4}
-_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split", 4: "tcgen05"}
+IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3, "tcgen05": 4, "tensorcore_lag2": 5}
+_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split", 4: "tcgen05",
+               5: "tensorcore_lag2"}
 STATUS = ["TTT_OK", "TTT_ERR_NULL", "TTT_ERR_SHAPE", "TTT_ERR_DTYPE", "TTT_ERR_ALIGN",
           "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT", "TTT_ERR_WORKSPACE"]
 
@@ -68,6 +70,8 @@ lib.ttt_linear_backward_workspace_size.restype = ctypes.c_size_t
 lib.ttt_linear_backward_workspace_size.argtypes = [_I] * 5
 lib.ttt_linear_backward.restype = _I
 lib.ttt_linear_backward.argtypes = [_I] * 7 + [_F] + [_P] * 20 + [ctypes.c_size_t, _P]
+lib.ttt_prologue_forward.restype = _I
+lib.ttt_prologue_forward.argtypes = [_I] * 6 + [_F, _F, _I] + [_P] * 10 + [_P]
 
 
 def linear_pick_impl(B, H, T, d, mini_batch, qkv_dtype, mode="ln") -> str:
@@ -426,3 +430,26 @@ def ttt_linear_backward(Q, K, V, eta, W0, b0, ln_gamma, ln_beta, dZ, dW_T=None, 
         _stream_handle(dev, stream))
     _check(st)
     return dQ, dK, dV, deta, dW0, db0, dgamma, dbeta
+
+
+def ttt_prologue_forward(x, theta_q, theta_k, theta_v, theta_lr, b_lr, *, pos0: int = 0,
+                         eta_base: float = 1.0, rope_base: float = 10000.0, rotary: bool = True,
+                         stream=None):
+    """The layer's prologue (see include/ttt.h): Q, K, V [B,H,T,d] bf16 and eta
+    [B,H,T] fp32 from x [B,T,d_model] bf16 and the bf16 weights."""
+    B, T, dm = x.shape
+    H, _, d = theta_q.shape
+    for name, t in (("x", x), ("theta_q", theta_q), ("theta_k", theta_k), ("theta_v", theta_v),
+                    ("theta_lr", theta_lr), ("b_lr", b_lr)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if any(t.dtype != torch.bfloat16 for t in (x, theta_q, theta_k, theta_v, theta_lr)) or b_lr.dtype != torch.float32:
+        raise TypeError("x and the weights must be bfloat16, b_lr float32")
+    dev = x.device
+    Q, K, V = (torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    eta = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    st = lib.ttt_prologue_forward(B, T, H, d, dm, int(pos0), float(eta_base), float(rope_base), int(bool(rotary)),
+                                  _ptr(x), _ptr(theta_q), _ptr(theta_k), _ptr(theta_v), _ptr(theta_lr), _ptr(b_lr),
+                                  _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _stream_handle(dev, stream))
+    _check(st)
+    return Q, K, V, eta

@@ -10,6 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libttt_b200.so")
+# the same library with the clock64 timeline stamps compiled in (timeline.py reads them)
+TIMELINE_LIB = os.path.join(PKG, "libttt_b200_timeline.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -28,22 +30,24 @@ def deps():
         os.path.join(ROOT, "include", "ttt.h")]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    stale = (not os.path.exists(LIB)) or any(os.path.getmtime(p) > os.path.getmtime(LIB) for p in deps())
+def build(force: bool = False, verbose: bool = False, timeline: bool = False) -> str:
+    out = TIMELINE_LIB if timeline else LIB
+    stale = (not os.path.exists(out)) or any(os.path.getmtime(p) > os.path.getmtime(out) for p in deps())
     if not (force or stale):
-        return LIB
+        return out
     nvcc = os.environ.get("NVCC", "nvcc")
     if not os.path.isabs(nvcc) and os.path.exists("/usr/local/cuda/bin/nvcc"):
         nvcc = "/usr/local/cuda/bin/nvcc"
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DTTT_TIMELINE"] if timeline else []), "-I", os.path.join(ROOT, "include"),
+           "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, timeline="--timeline" in sys.argv))

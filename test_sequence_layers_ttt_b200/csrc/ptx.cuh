@@ -160,9 +160,12 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
 }
 
 // Cheaper split for operands that are re-split every chunk: hi = x truncated to
-// bf16 (the top half of its bit pattern), lo = (x - hi) truncated to bf16; x - hi
-// is exact in fp32, so |x - hi - lo| < 2^-15 |x|.  Five instructions per pair:
-// two byte permutes, two masks and one packed fp32 subtraction.
+// bf16 (the top half of its bit pattern), lo = (x - hi) rounded to the nearest
+// bf16.  x - hi is exact in fp32 and below 2^-7 |x|, so |x - hi - lo| <= 2^-15 |x|
+// with no bias (a truncated lo would always shorten |x|, and that bias adds up
+// over the thousands of state updates of a long sequence).  Five instructions
+// per pair: a byte permute, two masks, one packed fp32 subtraction and one
+// packed conversion.
 __device__ __forceinline__ void split_pair_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
     hi = __byte_perm(b0, b1, 0x7632);
@@ -170,7 +173,8 @@ __device__ __forceinline__ void split_pair_trunc(float x0, float x1, uint32_t& h
     uint64_t d;
     asm("{\n .reg .b64 a, b;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %4};\n sub.rn.f32x2 %0, a, b;\n}\n"
         : "=l"(d) : "r"(b0), "r"(b1), "r"(t0), "r"(t1));
-    lo = __byte_perm((uint32_t)d, (uint32_t)(d >> 32), 0x7632);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(__uint_as_float((uint32_t)(d >> 32))),
+        "f"(__uint_as_float((uint32_t)d)));
 }
 // (x0, x1) += (y0, y1) as one packed fp32 add
 __device__ __forceinline__ void add2(float& x0, float& x1, float y0, float y1) {

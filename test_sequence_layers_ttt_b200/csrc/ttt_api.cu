@@ -50,7 +50,9 @@ bool prepare() {
     unsigned int stale = 0;
     return ttt::read_and_clear_device_error(&stale) == cudaSuccess &&
            ttt::read_and_clear_mlp_error(&stale) == cudaSuccess &&
-           ttt::read_and_clear_umma_error(&stale) == cudaSuccess;
+           ttt::read_and_clear_umma_error(&stale) == cudaSuccess &&
+           ttt::read_and_clear_hybrid_error(&stale) == cudaSuccess &&
+           ttt::read_and_clear_prologue_error(&stale) == cudaSuccess;
 }
 
 bool valid_mini_batch(int mb) { return mb >= 1 && (mb % 16 == 0 || mb == 1 || mb == 2 || mb == 4 || mb == 8); }
@@ -73,11 +75,13 @@ ttt_status finish(cudaError_t launch, cudaStream_t stream) {
     if (launch != cudaSuccess) return TTT_ERR_CUDA;
     if (!check_env()) return TTT_OK;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
-    unsigned int flag = 0, mlp_flag = 0, umma_flag = 0;
+    unsigned int flag = 0, mlp_flag = 0, umma_flag = 0, hyb_flag = 0, pro_flag = 0;
     if (ttt::read_and_clear_device_error(&flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_mlp_error(&mlp_flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_umma_error(&umma_flag) != cudaSuccess) return TTT_ERR_CUDA;
-    return (flag | mlp_flag | umma_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
+    if (ttt::read_and_clear_hybrid_error(&hyb_flag) != cudaSuccess) return TTT_ERR_CUDA;
+    if (ttt::read_and_clear_prologue_error(&pro_flag) != cudaSuccess) return TTT_ERR_CUDA;
+    return (flag | mlp_flag | umma_flag | hyb_flag | pro_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
 }
 
 ttt_status validate_linear(const LinearArgs& a) {
@@ -206,9 +210,40 @@ ttt_status validate_linear_backward(const ttt::LinearBwdArgs& a, const void* wor
     return check_aliasing(outs, 8, ins, same_as, 12);
 }
 
+ttt_status validate_prologue(const ttt::PrologueArgs& a) {
+    if (a.B < 1 || a.T < 1 || a.H < 1 || a.d_model < 1 || (long long)a.B * a.T >= (1LL << 31)) return TTT_ERR_SHAPE;
+    if (!(a.rope_base > 1.f) || !(a.eta_base == a.eta_base)) return TTT_ERR_SHAPE;
+    if (!ttt::prologue_supports(a.B, a.T, a.H, a.d, a.d_model)) return TTT_ERR_UNSUPPORTED;
+    const void* req[] = {a.x, a.theta_q, a.theta_k, a.theta_v, a.theta_lr, a.b_lr, a.Q, a.K, a.V, a.eta};
+    for (const void* p : req)
+        if (!p) return TTT_ERR_NULL;
+    for (const void* p : req)
+        if (!aligned16(p)) return TTT_ERR_ALIGN;
+    const size_t tok = (size_t)a.B * a.T, hd = (size_t)a.H * a.d, w = (size_t)a.d_model * hd * 2;
+    Span ins[] = {{a.x, tok * a.d_model * 2}, {a.theta_q, w}, {a.theta_k, w}, {a.theta_v, w},
+                  {a.theta_lr, (size_t)a.H * a.d_model * 2}, {a.b_lr, (size_t)a.H * 4}};
+    Span outs[] = {{a.Q, tok * hd * 2}, {a.K, tok * hd * 2}, {a.V, tok * hd * 2}, {a.eta, tok * a.H * 4}};
+    const int same_as[] = {-1, -1, -1, -1};
+    return check_aliasing(outs, 4, ins, same_as, 6);
+}
+
 }  // namespace
 
 extern "C" {
+
+ttt_status ttt_prologue_forward(int B, int T, int H, int d, int d_model, int pos0, float eta_base,
+                                float rope_base, int rotary, const void* x, const void* theta_q,
+                                const void* theta_k, const void* theta_v, const void* theta_lr,
+                                const float* b_lr, void* Q, void* K, void* V, float* eta,
+                                ttt_stream_t stream) {
+    ttt::PrologueArgs a{B, T, H, d, d_model, pos0, rotary ? 1 : 0, eta_base, rope_base, x, theta_q, theta_k,
+                        theta_v, theta_lr, b_lr, Q, K, V, eta};
+    ttt_status st = validate_prologue(a);
+    if (st != TTT_OK) return st;
+    if (!prepare()) return TTT_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return finish(ttt::launch_prologue(a, s), s);
+}
 
 size_t ttt_linear_backward_workspace_size(int B, int H, int T, int d, int mini_batch) {
     return ttt::linear_backward_workspace_bytes(B, H, T, d, mini_batch);
@@ -266,6 +301,9 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, t
         case TTT_IMPL_TCGEN05:
             if (!ttt::linear_umma_supports(a)) return TTT_ERR_UNSUPPORTED;
             return finish(ttt::launch_linear_umma(a, s), s);
+        case TTT_IMPL_TENSORCORE_LAG2:
+            if (!ttt::linear_hybrid_supports(a)) return TTT_ERR_UNSUPPORTED;
+            return finish(ttt::launch_linear_hybrid(a, s), s);
         default:
             return TTT_ERR_UNSUPPORTED;
     }
@@ -398,11 +436,24 @@ const char* ttt_status_string(ttt_status status) {
         case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED: shape, mode or kernel family not built";
         case TTT_ERR_CUDA: return "TTT_ERR_CUDA: CUDA launch or execution error";
         case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT: a kernel abandoned a bounded wait";
-        case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE: workspace missing or smaller than required";
+        case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE: workspace missing or too small for these arguments";
         default: return "TTT_ERR_UNKNOWN";
     }
 }
 
 int ttt_abi_version(void) { return 102; }
+
+#ifdef TTT_TIMELINE
+// Timeline builds only (not part of the ABI): copy the clock64 stamps of CTA 0
+// of the last launch of kernel `which` (0: ttt_linear_lag_kernel, 1:
+// ttt_linear_hybrid_kernel) into out[kTlRoles][kTlChunks][kTlEvents].
+int ttt_debug_timeline(int which, long long* out) {
+    if (!out) return TTT_ERR_NULL;
+    if (cudaDeviceSynchronize() != cudaSuccess) return TTT_ERR_CUDA;
+    const cudaError_t e = which == 0 ? ttt::read_lag_timeline(out) : which == 1 ? ttt::read_hybrid_timeline(out)
+                                                                              : cudaErrorInvalidValue;
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

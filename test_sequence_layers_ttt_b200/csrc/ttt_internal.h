@@ -47,6 +47,12 @@ bool linear_umma_supports(const LinearArgs& a);
 cudaError_t launch_linear_umma(const LinearArgs& a, cudaStream_t stream);
 cudaError_t read_and_clear_umma_error(unsigned int* out);
 
+// Lag-2 scan: the state increment on tcgen05, the W products and the chain on mma.sync
+// (ttt_linear_hybrid.cu); same shapes as linear_tc.
+bool linear_hybrid_supports(const LinearArgs& a);
+cudaError_t launch_linear_hybrid(const LinearArgs& a, cudaStream_t stream);
+cudaError_t read_and_clear_hybrid_error(unsigned int* out);
+
 // Decode with the state in registers (d = 64); in place on W_T / b_T and Wm_T / bm_T.
 bool linear_decode_supports(const LinearArgs& a);
 cudaError_t launch_linear_decode(const LinearArgs& a, cudaStream_t stream);
@@ -61,6 +67,19 @@ struct LinearBwdArgs {
 bool linear_backward_supports(const LinearBwdArgs& a);
 size_t linear_backward_workspace_bytes(int B, int H, int T, int d, int mini_batch);
 cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cudaStream_t stream);
+
+// The layer's prologue (ttt_prologue.cu): projections, learning-rate gate, rotary embedding.
+struct PrologueArgs {
+    int B, T, H, d, d_model, pos0, rotary;
+    float eta_base, rope_base;
+    const void *x, *theta_q, *theta_k, *theta_v, *theta_lr;
+    const float* b_lr;
+    void *Q, *K, *V;
+    float* eta;
+};
+bool prologue_supports(int B, int T, int H, int d, int d_model);
+cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
+cudaError_t read_and_clear_prologue_error(unsigned int* out);
 
 bool mlp_generic_supports(const MlpArgs& a);
 cudaError_t launch_mlp_generic(const MlpArgs& a, cudaStream_t stream);
@@ -79,6 +98,10 @@ cudaError_t read_and_clear_mlp_error(unsigned int* out);
 
 // Device-side error word set by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_device_error(unsigned int* out);
+#ifdef TTT_TIMELINE
+cudaError_t read_lag_timeline(long long* out);     // kTlRoles x kTlChunks x kTlEvents stamps
+cudaError_t read_hybrid_timeline(long long* out);
+#endif
 
 // Fault-injection hook: the chunk index named by TTT_DEBUG_DROP_CHUNK (read once
 // per process), whose loads the tensor-core TTT-Linear producer skips; -1 when unset.

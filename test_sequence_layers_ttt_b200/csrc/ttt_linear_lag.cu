@@ -34,6 +34,9 @@
 //   PB  warp 14     M_c and A_c (16 x 16 tensor-core products, eta folded in)
 // Every product with an fp32 operand splits it into bf16 hi + lo terms
 // (relative error below 2^-15); bf16 inputs are exact; accumulation is fp32.
+// The state is kept centred on its per-input-row means over the output
+// features (added back to W_T, b_T at the end), so y = x W + b has a mean near
+// zero and the one-pass LayerNorm variance does not cancel.
 // The W-free inputs run up to NPRE chunks ahead in a ring, and Q~W~ is handed
 // to the output warps through four buffers, so the slower output path does
 // not hold back the chain's inputs.
@@ -44,6 +47,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "timeline.cuh"
 #include "tma_host.h"
 #include "ttt_internal.h"
 
@@ -51,6 +55,8 @@ namespace ttt {
 
 // set by kernels that abandon a bounded wait; read (and cleared) by the host with TTT_CHECK=1
 __device__ unsigned int g_ttt_error_word = 0;
+
+TTT_TIMELINE_BUFFER(g_lag_timeline);  // roles: 0 CH, 1 WP, 2 OW, 3 PR, 4 PA, 5 PB
 
 namespace {
 
@@ -84,6 +90,7 @@ struct LagSmem {
     float red_ch[2][kChunk][5][4];          // [buf][tok][sum][warp]
     float red_ow[2][kChunk][12];            // [buf][tok][2 sums x 4 warps + pad]
     float gam[D], bet[D];
+    float u[D + 1];                         // per-input-row means removed from the state (row D: bias)
     uint64_t in_full[NS], in_empty[NS];
     uint64_t pre_full[NPRE], pre_empty[NPRE], p_full[2], p_empty[2];
     uint64_t g_full[2], g_empty[2], qw_full[4], qw_empty[4];
@@ -133,6 +140,8 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const int bh = blockIdx.x, h = bh % H;
     const int n = T / kChunk;
     volatile int* abort_flag = &s.abort_flag;
+    const bool tl_lead = (tid & 31) == 0 && (warp == 0 || warp == kWarpWP0 || warp == kWarpOW0 || warp >= kWarpPR);
+    (void)tl_lead;
 
     if (tid < D) {
         s.gam[tid] = gamma[h * D + tid];
@@ -172,7 +181,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             int issued = 0;
             for (int c = 0; c < n; c++) {
                 const int slot = c % NS;
+                TTT_STAMP(g_lag_timeline, tl_lead, 3, c, 0);
                 if (c >= NS && !wait_bounded(&s.in_empty[slot], ((c / NS) - 1) & 1, abort_flag)) break;
+                TTT_STAMP(g_lag_timeline, tl_lead, 3, c, 1);
                 if (c == drop_chunk) continue;  // fault-injection hook: this chunk is never loaded
                 ptx::mbar_arrive_expect_tx(&s.in_full[slot], kStageTx);
                 ptx::tma_load_3d(s.K[slot], &tmK, &s.in_full[slot], 0, c * kChunk, bh);
@@ -199,8 +210,11 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     if (warp == kWarpPA) {
         for (int c = 0; c < n; c++) {
             const int slot = c % NS, b = c % NPRE;
+            TTT_STAMP(g_lag_timeline, tl_lead, 4, c, 0);
             wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 4, c, 1);
             if (c >= NPRE) wait_use(&s.pre_empty[b], c / NPRE - 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 4, c, 2);
             float rs0 = 0.f, rs1 = 0.f;  // row g, row g + 8
 #pragma unroll
             for (int w = 0; w < kCH; w++) {
@@ -232,6 +246,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             if (lane < kChunk) s.etac[b][lane] = s.eta[slot][lane];
             arrive1(&s.pre_full[b], lane);
             arrive1(&s.in_empty[slot], lane);
+            TTT_STAMP(g_lag_timeline, tl_lead, 4, c, 3);
         }
         return;
     }
@@ -240,8 +255,11 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     if (warp == kWarpPB) {
         for (int c = 0; c < n; c++) {
             const int slot = c % NS, b = c % NPRE;
+            TTT_STAMP(g_lag_timeline, tl_lead, 5, c, 0);
             wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 5, c, 1);
             if (c >= NPRE) wait_use(&s.pre_empty[b], c / NPRE - 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 5, c, 2);
             const uint32_t xs = ptx::smem_addr(s.K[slot]);
             const uint32_t qs = ptx::smem_addr(s.Q[slot]);
             const int mi = lane >> 3;
@@ -299,6 +317,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             s.afrag[b][1][lane] = make_uint4(al[0], al[1], al[2], al[3]);
             arrive1(&s.pre_full[b], lane);
             if (c > 0) arrive1(&s.in_empty[pslot], lane);  // last use of X_{c-1}, eta_{c-1}
+            TTT_STAMP(g_lag_timeline, tl_lead, 5, c, 3);
         }
         if (n > 0) arrive1(&s.in_empty[(n - 1) % NS], lane);
         return;
@@ -308,20 +327,39 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     if (warp >= kWarpWP0 && warp < kWarpOW0) {
         const int w = warp - kWarpWP0;
         const float* W0b = W0 + (size_t)bh * D * D;
+        // The state is kept centred on its per-input-row means over the output
+        // features (and b on its mean): every row of G sums to zero, so the update
+        // leaves these means unchanged, and LayerNorm ignores the per-token shift
+        // they add to x W + b.  With y centred, the one-pass variance of the chain
+        // and output statistics does not cancel.  The means are added back at the end.
+        {
+            const int st = tid - kWarpWP0 * 32;
+            if (st < D) {
+                float acc = 0.f;
+                for (int j = 0; j < D; j++) acc += W0b[st * D + j];
+                s.u[st] = acc * (1.f / D);
+            } else if (st == D) {
+                float acc = 0.f;
+                for (int j = 0; j < D; j++) acc += b0[(size_t)bh * D + j];
+                s.u[D] = acc * (1.f / D);
+            }
+            ptx::named_bar_sync(3, kWP * 32);
+        }
         float Wt[8][4];  // W^T rows 16w+g (+8), input columns 8j + 2t (+1)
 #pragma unroll
         for (int jj = 0; jj < 8; jj++) {
             const int in0 = 8 * jj + 2 * t;
-            Wt[jj][0] = W0b[in0 * D + 16 * w + g];
-            Wt[jj][1] = W0b[(in0 + 1) * D + 16 * w + g];
-            Wt[jj][2] = W0b[in0 * D + 16 * w + 8 + g];
-            Wt[jj][3] = W0b[(in0 + 1) * D + 16 * w + 8 + g];
+            const float u0 = s.u[in0], u1 = s.u[in0 + 1];
+            Wt[jj][0] = W0b[in0 * D + 16 * w + g] - u0;
+            Wt[jj][1] = W0b[(in0 + 1) * D + 16 * w + g] - u1;
+            Wt[jj][2] = W0b[in0 * D + 16 * w + 8 + g] - u0;
+            Wt[jj][3] = W0b[(in0 + 1) * D + 16 * w + 8 + g] - u1;
         }
         // bias column (x~ has a trailing 1): accumulator tile whose column 0 is b
         float Bt[4] = {0.f, 0.f, 0.f, 0.f};
         if (t == 0) {
-            Bt[0] = b0[(size_t)bh * D + 16 * w + g];
-            Bt[2] = b0[(size_t)bh * D + 16 * w + 8 + g];
+            Bt[0] = b0[(size_t)bh * D + 16 * w + g] - s.u[D];
+            Bt[2] = b0[(size_t)bh * D + 16 * w + 8 + g] - s.u[D];
         }
         const uint32_t ones = g == 0 ? kOnesBf16x2 : 0u;
 
@@ -374,7 +412,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         for (int j = 1; j <= n; j++) {
             // ---- update with G_{j-1}: W~_j = W~_{j-1} - X~_{j-1}^T diag(eta_{j-1}) G_{j-1}
             const int pb = (j - 1) & 1, pslot = (j - 1) % NS;
+            TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 0);
             wait_use(&s.g_full[pb], (j - 1) >> 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 1);
             uint32_t ah[4], al[4];  // -(eta G)^T: rows = features 16w.., k = tokens
             {
                 const int mi = lane >> 3, row = (mi >> 1) * 8 + (lane & 7), chunk = 2 * w + (mi & 1);
@@ -412,23 +452,29 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             }
             arrive1(&s.g_empty[pb], lane);
             arrive1(&s.in_empty[pslot], lane);
+            TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 2);
             if (j == n) break;
 
             split_w();
+            TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 3);
             // ---- P_{j+1} = X~_{j+1} W~_j
             if (j + 1 < n) {
                 const int nb = (j + 1) & 1, nslot = (j + 1) % NS;
                 wait_bounded(&s.in_full[nslot], ((j + 1) / NS) & 1, abort_flag);
                 if (j + 1 >= 2) wait_use(&s.p_empty[nb], ((j + 1) >> 1) - 1, abort_flag);
+                TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 4);
                 product(ptx::smem_addr(s.K[nslot]), s.pbuf[nb][w][lane]);
                 arrive1(&s.p_full[nb], lane);
+                TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 5);
             }
             // ---- Q~_j W~_j for the output warps
             {
                 const int qb = j & 3;
                 if (j >= 4) wait_use(&s.qw_empty[qb], (j >> 2) - 1, abort_flag);
+                TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 6);
                 product(ptx::smem_addr(s.Q[j % NS]), s.qwbuf[qb][w][lane]);
                 arrive1(&s.qw_full[qb], lane);
+                TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 7);
             }
         }
 
@@ -437,14 +483,15 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 #pragma unroll
         for (int jj = 0; jj < 8; jj++) {
             const int in0 = 8 * jj + 2 * t;
-            WTb[in0 * D + 16 * w + g] = Wt[jj][0];
-            WTb[(in0 + 1) * D + 16 * w + g] = Wt[jj][1];
-            WTb[in0 * D + 16 * w + 8 + g] = Wt[jj][2];
-            WTb[(in0 + 1) * D + 16 * w + 8 + g] = Wt[jj][3];
+            const float u0 = s.u[in0], u1 = s.u[in0 + 1];
+            WTb[in0 * D + 16 * w + g] = Wt[jj][0] + u0;
+            WTb[(in0 + 1) * D + 16 * w + g] = Wt[jj][1] + u1;
+            WTb[in0 * D + 16 * w + 8 + g] = Wt[jj][2] + u0;
+            WTb[(in0 + 1) * D + 16 * w + 8 + g] = Wt[jj][3] + u1;
         }
         if (t == 0) {
-            b_T[(size_t)bh * D + 16 * w + g] = Bt[0];
-            b_T[(size_t)bh * D + 16 * w + 8 + g] = Bt[2];
+            b_T[(size_t)bh * D + 16 * w + g] = Bt[0] + s.u[D];
+            b_T[(size_t)bh * D + 16 * w + 8 + g] = Bt[2] + s.u[D];
         }
         return;
     }
@@ -503,6 +550,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         }
         for (int c = 0; c < n; c++) {
             const int b = c & 1;
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 0);
             float y[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; nt++)
@@ -516,7 +564,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 ptx::mma_bf16(y[0], ml.x, ml.y, ml.z, ml.w, gbh[0], gbh[1]);
                 ptx::mma_bf16(y[1], ml.x, ml.y, ml.z, ml.w, gbh[2], gbh[3]);
             }
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 1);
             if (c + 1 < n) load_pre(c + 1);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 2);
             const float* gcc = gcv;
             const float* c0c = c0v;
 
@@ -551,6 +601,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     for (int q = 0; q < 5; q++) s.red_ch[b][8 * rh + g][q][w] = sm[rh][q];
             }
             ptx::named_bar_sync(1, kCH * 32);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 3);
 
             float G[2][2][2];  // [rh][nt][e]
 #pragma unroll
@@ -588,7 +639,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     gbl[2 * nt + rh] = ptx::movmatrix_t(lo);
                 }
             // G_c and -eta G_c (hi/lo) -> shared tiles for the state and output warps
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 4);
             if (c >= 2) wait_use(&s.g_empty[b], (c >> 1) - 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 5);
 #pragma unroll
             for (int rh = 0; rh < 2; rh++)
 #pragma unroll
@@ -604,7 +657,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 }
             __syncwarp();  // every lane's tile stores before the hand-off
             if (lane == 0) ptx::mbar_arrive(&s.g_full[b]);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 6);
             if (c + 1 < n) load_inputs(c + 1);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 7);
         }
         return;
     }
@@ -624,7 +679,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         for (int c = 0; c < n; c++) {
             const int b = c & 1, slot = c % NS;
             float z[2][4];
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 0);
             wait_use(&s.qw_full[c & 3], c >> 2, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 1);
             {
                 const float4 p0 = s.qwbuf[c & 3][w][lane][0], p1 = s.qwbuf[c & 3][w][lane][1];
                 z[0][0] = p0.x; z[0][1] = p0.y; z[0][2] = p0.z; z[0][3] = p0.w;
@@ -634,7 +691,9 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             wait_use(&s.pre_full[c % NPRE], c / NPRE, abort_flag);
             const uint4 ah = s.afrag[c % NPRE][0][lane], al = s.afrag[c % NPRE][1][lane];
             arrive1(&s.pre_empty[c % NPRE], lane);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 2);
             wait_use(&s.g_full[b], c >> 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 3);
             {
                 const int mi = lane >> 3, row = (mi & 1) * 8 + (lane & 7), chunk = 2 * w + (mi >> 1);
                 uint32_t gh0, gh1, gh2, gh3, gl0, gl1, gl2, gl3;
@@ -672,8 +731,11 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 for (int rh = 0; rh < 2; rh++)
                     *reinterpret_cast<float2*>(&s.red_ow[b][8 * rh + g][2 * w]) = make_float2(ps[rh][0], ps[rh][1]);
             }
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 4);
             ptx::named_bar_sync(2, kOW * 32);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 5);
             wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 6);
 #pragma unroll
             for (int rh = 0; rh < 2; rh++) {
                 const int row = 8 * rh + g;
@@ -695,6 +757,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 }
             }
             arrive1(&s.in_empty[slot], lane);
+            TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 7);
         }
     }
 }
@@ -728,6 +791,12 @@ cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream) {
                                                            a.beta, a.Z, a.W_T, a.b_T, drop_chunk_hook());
     return cudaPeekAtLastError();
 }
+
+#ifdef TTT_TIMELINE
+cudaError_t read_lag_timeline(long long* out) {
+    return cudaMemcpyFromSymbol(out, g_lag_timeline, sizeof(g_lag_timeline));
+}
+#endif
 
 cudaError_t read_and_clear_device_error(unsigned int* out) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_ttt_error_word, sizeof(unsigned int));

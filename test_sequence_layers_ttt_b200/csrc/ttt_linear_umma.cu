@@ -38,8 +38,8 @@
 //   PA  14    gamma * (x + beta - v) per (feature, token) and its row sums.
 //   PB  15    S1 (as mma B fragments), S2 and L (as hi/lo operand tiles).
 // Precision: every product with an fp32 operand splits it into bf16 hi + lo
-// (hi the truncated top half, lo the truncated remainder: |x - hi - lo| below
-// 2^-15 |x|) and drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
+// (hi the truncated top half, lo the remainder rounded to nearest: |x - hi - lo|
+// at most 2^-15 |x|, unbiased) and drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
 // and added to the fp32 registers with fp32 adds (tensor-core accumulation of
 // thousands of increments would not round to nearest).
 // Feature order: accumulator row r = 16 j + i holds output feature
