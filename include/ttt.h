@@ -316,6 +316,39 @@ ttt_status ttt_linear_backward(int B, int H, int T, int d, int mini_batch, ttt_d
                                float* deta, float* dW0, float* db0, float* dgamma, float* dbeta,
                                void* workspace, size_t workspace_bytes, ttt_stream_t stream);
 
+/*
+ * ttt_linear_backward without a workspace argument, for callers that cannot
+ * allocate device memory: for example a host program whose own allocator owns
+ * all device memory and grants a library nothing at call time, or a loop with a
+ * latency budget that an allocation (and the synchronisation it may bring)
+ * would break.  The pages define no such call; it exists only for this reason.
+ *   The workspace is a fixed array inside the library,
+ *   TTT_BACKWARD_STATIC_WORKSPACE_BYTES (32 MiB) long, which every GPU that
+ *   loads the library holds until the process exits.  Arguments whose
+ *   ttt_linear_backward_workspace_size exceeds it return TTT_ERR_WORKSPACE
+ *   before anything runs (for d = 64 it holds about 2000 mini-batch states,
+ *   summed over batch and heads).
+ *   The call allocates nothing: no cudaMalloc, no library allocator.  The
+ *   first call on a device looks up the array's device address (one
+ *   cudaGetSymbolAddress with that device current) and keeps it; make that
+ *   first call before any stream capture.
+ *   Every call on a device shares the one array, and the array keeps the last
+ *   call's contents; the kernels write every word of it they later read, so
+ *   nothing needs to start at zero.  Calls that may overlap on the GPU (on
+ *   several streams, or from several host threads) race on it: run them one
+ *   after another.
+ *   Arguments, outputs and errors otherwise as ttt_linear_backward.
+ */
+#define TTT_BACKWARD_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+ttt_status ttt_linear_backward_static(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                                      ttt_mode mode, float ln_eps, const void* Q, const void* K,
+                                      const void* V, const float* eta, const float* W0, const float* b0,
+                                      const float* ln_gamma, const float* ln_beta, const float* dZ,
+                                      const float* dW_T, const float* db_T, float* dQ, float* dK,
+                                      float* dV, float* deta, float* dW0, float* db0, float* dgamma,
+                                      float* dbeta, ttt_stream_t stream);
+
 /* Static string naming a status code; never NULL. */
 const char* ttt_status_string(ttt_status status);
 

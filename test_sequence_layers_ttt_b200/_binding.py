@@ -70,6 +70,9 @@ lib.ttt_linear_backward_workspace_size.restype = ctypes.c_size_t
 lib.ttt_linear_backward_workspace_size.argtypes = [_I] * 5
 lib.ttt_linear_backward.restype = _I
 lib.ttt_linear_backward.argtypes = [_I] * 7 + [_F] + [_P] * 20 + [ctypes.c_size_t, _P]
+lib.ttt_linear_backward_static.restype = _I
+lib.ttt_linear_backward_static.argtypes = [_I] * 7 + [_F] + [_P] * 19 + [_P]
+STATIC_WORKSPACE_BYTES = 32 << 20  # TTT_BACKWARD_STATIC_WORKSPACE_BYTES in include/ttt.h
 lib.ttt_prologue_forward.restype = _I
 lib.ttt_prologue_forward.argtypes = [_I] * 6 + [_F, _F, _I] + [_P] * 10 + [_P]
 

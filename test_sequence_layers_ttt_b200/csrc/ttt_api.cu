@@ -425,6 +425,22 @@ ttt_status ttt_mlp_forward(int B, int H, int T, int d, int hidden, int mini_batc
                                 TTT_IMPL_AUTO, stream);
 }
 
+ttt_status ttt_linear_backward_static(int B, int H, int T, int d, int mini_batch, ttt_dtype qkv_dtype,
+                                      ttt_mode mode, float ln_eps, const void* Q, const void* K, const void* V,
+                                      const float* eta, const float* W0, const float* b0, const float* ln_gamma,
+                                      const float* ln_beta, const float* dZ, const float* dW_T, const float* db_T,
+                                      float* dQ, float* dK, float* dV, float* deta, float* dW0, float* db0,
+                                      float* dgamma, float* dbeta, ttt_stream_t stream) {
+    // the size check comes first: shapes beyond the fixed array are refused before any CUDA call
+    const size_t need = ttt::linear_backward_workspace_bytes(B, H, T, d, mini_batch);
+    if (need > ttt::kBackwardStaticWorkspaceBytes) return TTT_ERR_WORKSPACE;
+    float* ws = ttt::backward_static_workspace();
+    if (!ws) return TTT_ERR_CUDA;
+    return ttt_linear_backward(B, H, T, d, mini_batch, qkv_dtype, mode, ln_eps, Q, K, V, eta, W0, b0, ln_gamma,
+                               ln_beta, dZ, dW_T, db_T, dQ, dK, dV, deta, dW0, db0, dgamma, dbeta, ws,
+                               ttt::kBackwardStaticWorkspaceBytes, stream);
+}
+
 const char* ttt_status_string(ttt_status status) {
     switch (status) {
         case TTT_OK: return "TTT_OK";

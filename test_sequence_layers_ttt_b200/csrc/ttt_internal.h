@@ -64,6 +64,9 @@ struct LinearBwdArgs {
     const float *dZ, *dW_T, *db_T;
     float *dQ, *dK, *dV, *deta, *dW0, *db0, *dgamma, *dbeta;
 };
+// Size of the file-scope workspace of ttt_linear_backward_static (TTT_BACKWARD_STATIC_WORKSPACE_BYTES).
+constexpr size_t kBackwardStaticWorkspaceBytes = TTT_BACKWARD_STATIC_WORKSPACE_BYTES;
+float* backward_static_workspace();
 bool linear_backward_supports(const LinearBwdArgs& a);
 size_t linear_backward_workspace_bytes(int B, int H, int T, int d, int mini_batch);
 cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cudaStream_t stream);

@@ -24,10 +24,18 @@
 //   3. ttt_linear_dgamma_kernel sums the per-(batch, head) gamma / beta
 //      partials over the batch in a fixed order (deterministic).
 // One mini-batch is processed at a time (mini_batch <= 16 tokens).
+#include <atomic>
+
 #include "common.cuh"
 #include "ttt_internal.h"
 
 namespace ttt {
+
+// Workspace of ttt_linear_backward_static: a fixed array that every device
+// loading the library holds until the process exits, for callers that cannot
+// allocate device memory.  Shared by every call on a device.
+static __device__ __align__(256) unsigned char g_backward_static_workspace[kBackwardStaticWorkspaceBytes];
+
 namespace {
 
 constexpr int kBwdThreads = 256;
@@ -473,6 +481,27 @@ cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cud
     const int hd = f.H * f.d;
     ttt_linear_dgamma_kernel<<<(hd + 255) / 256, 256, 0, stream>>>(f.B, f.H, f.d, gb, a.dgamma, a.dbeta);
     return cudaPeekAtLastError();
+}
+
+}  // namespace ttt
+
+namespace ttt {
+
+// Device address of the static workspace on the current device.  Host code
+// cannot use the array's name as a device pointer; cudaGetSymbolAddress gives
+// the address, once per device (with that device current), cached for later
+// calls.  Returns nullptr if the runtime reports an error.
+float* backward_static_workspace() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<void*> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_backward_static_workspace) != cudaSuccess) return nullptr;
+        cache[dev].store(p, std::memory_order_release);
+    }
+    return static_cast<float*>(p);
 }
 
 }  // namespace ttt
