@@ -87,14 +87,14 @@ KERNEL_SOURCES = {
     "ttt_linear_lag_kernel": ("ttt_linear_lag.cu", "ptx.cuh", "common.cuh", "tma_host.h", "ttt_internal.h"),
     "ttt_linear_umma_kernel": ("ttt_linear_umma.cu", "ptx.cuh", "tcgen05.cuh", "common.cuh", "tma_host.h",
                                "ttt_internal.h"),
-    "ttt_linear_hybrid_kernel": ("ttt_linear_hybrid.cu", "ptx.cuh", "tcgen05.cuh", "common.cuh", "tma_host.h",
-                                 "ttt_internal.h"),
     "ttt_linear_generic_kernel": ("ttt_linear_generic.cu", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_tc_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_split_kernel": ("ttt_mlp_tc.cu", "ptx.cuh", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_generic_kernel": ("ttt_mlp_generic.cu", "common.cuh", "ttt_internal.h"),
     "ttt_linear_decode_kernel": ("ttt_linear_decode.cu", "common.cuh", "ttt_internal.h"),
     "ttt_mlp_decode_kernel": ("ttt_mlp_decode.cu", "common.cuh", "ttt_internal.h"),
+    "ttt_prologue_kernel": ("ttt_prologue.cu", "ptx.cuh", "tcgen05.cuh", "common.cuh", "tma_host.h",
+                            "ttt_internal.h"),
 }
 
 
@@ -118,8 +118,8 @@ def recorded_traffic(kernel: str, workload: str):
         return None
     with open(path) as fh:
         for line in fh:
-            f = line.split()
-            if len(f) == 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
+            f = line.split("#")[0].split()
+            if len(f) == 4 and f[0] == kernel and f[1] == workload:
                 return int(f[3]) if f[2] == kernel_source_hash(kernel) else None
     return None
 
@@ -293,10 +293,39 @@ def cpu_oracle_decode_sample(w, inp, target_s: float):
                       f"float64 primal oracle, {dt:.2f} s"}
 
 
+def run_reference_prologue(args):
+    p = PROLOGUE
+    host = prologue_inputs(args.seed, p["B"], p["T"], p["H"], p["d"], p["d_model"])
+    for _ in range(args.warmup):
+        cpu_oracle_prologue_sample(p, host, 0.5)
+    vals, r = [], None
+    t_start = time.perf_counter()
+    per_step = min(args.ref_seconds, 150.0 / max(args.steps, 1))
+    for _ in range(args.steps):
+        r = cpu_oracle_prologue_sample(p, host, per_step)
+        vals.append(r["value"])
+    elapsed = time.perf_counter() - t_start
+    value = statistics.median(vals)
+    print(json.dumps({
+        "impl": "reference", "metric": "TTT prologue tokens/sec on 1 B200 (1.3B layer: d_model 2048, 32 heads of "
+                                       "64, 32k ctx); % of tensor roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": p["name"], "B": p["B"], "T": p["T"], "H": p["H"], "d": p["d"],
+                   "d_model": p["d_model"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0}), flush=True)
+
+
 def run_reference(args, world, rank):
-    w = WORKLOADS[args.workload]
     if rank != 0:
         return
+    if args.workload == PROLOGUE["name"]:
+        return run_reference_prologue(args)
+    w = WORKLOADS[args.workload]
     inp = make_inputs(w, args.seed)
     sample = cpu_oracle_decode_sample if args.workload in DECODE_WORKLOADS else cpu_oracle_sample
     for _ in range(args.warmup):
@@ -484,9 +513,138 @@ def run_decode(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# The layer's prologue on the 1.3B-layer shape: x [2, 32768, 2048] bf16 against the
+# Q/K/V and learning-rate weights of 32 heads of d = 64.
+PROLOGUE = {"name": "prologue_1p3b_32k", "B": 2, "T": 32768, "H": 32, "d": 64, "d_model": 2048}
+
+
+def prologue_inputs(seed: int, B: int, T: int, H: int, d: int, d_model: int):
+    """Seeded synthetic prologue inputs: x ~ N(0, 1), every weight ~ N(0, 1/d_model)
+    (bf16); b_lr ~ N(0, 1) fp32."""
+    g = torch.Generator().manual_seed(seed)
+    bf = lambda *shape, std: (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+    x = bf(B, T, d_model, std=1.0)
+    tq, tk, tv = (bf(H, d_model, d, std=d_model ** -0.5) for _ in range(3))
+    tl = bf(H, d_model, std=d_model ** -0.5)
+    bl = torch.randn(H, generator=g)
+    return x, tq, tk, tv, tl, bl
+
+
+def prologue_flops(p) -> int:
+    """2 M d_model N with M = B T tokens and N = 3 H d + H output columns."""
+    return 2 * p["B"] * p["T"] * p["d_model"] * (3 * p["H"] * p["d"] + p["H"])
+
+
+def cpu_oracle_prologue_sample(p, host, target_s: float):
+    """Time the float64 prologue oracle on the first tokens of batch 0, as many
+    as fit in about target_s seconds; tokens/s."""
+    import oracle.prologue as op
+    x, tq, tk, tv, tl, bl = host
+    n, dt = 16, 0.0
+    while True:
+        t0 = time.perf_counter()
+        op.project(x[:1, :n], tq, tk, tv, tl, bl)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or n >= p["T"]:
+            break
+        n = min(p["T"], n * 4)
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of one sequence, all {p['H']} heads, float64 oracle (numpy einsum, one "
+                      f"thread), {dt:.2f} s"}
+
+
+def run_prologue(args, world, rank, local):
+    """Forward tokens/s of ttt_prologue_forward on the 1.3B-layer shape."""
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+
+    p = PROLOGUE
+    dev = torch.device("cuda", local)
+    host = prologue_inputs(args.seed + rank, p["B"], p["T"], p["H"], p["d"], p["d_model"])
+    g = [t.to(dev) for t in host]
+    B, T, H, d = p["B"], p["T"], p["H"], p["d"]
+    Q, K, V = (torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    eta = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x):
+        st = ttt.lib.ttt_prologue_forward(B, T, H, d, p["d_model"], 0, 1.0, 10000.0, 1, ttt._ptr(x),
+                                          *(ttt._ptr(t) for t in g[1:]), ttt._ptr(Q), ttt._ptr(K), ttt._ptr(V),
+                                          ttt._ptr(eta), ttt._stream_handle(dev, stream))
+        ttt._check(st)
+
+    for _ in range(args.warmup):
+        step(g[0])
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(g[0])
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    ms_per_step = dist_max(start.elapsed_time(end), world) / args.steps
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    value = B * T * world / (ms_per_step * 1e-3)
+
+    # end to end: x from pinned host memory, Q/K/V/eta back to pinned host memory
+    x_host = host[0].pin_memory()
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (Q, K, V, eta)]
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+    x_dev = torch.empty_like(g[0])
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        for o, t in zip(outs_host, (Q, K, V, eta)):
+            o.copy_(t, non_blocking=True)
+        stream.synchronize()
+    e2e_s = dist_max((time.perf_counter() - t0) / e2e_steps, world)
+
+    cpu_base = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_prologue_sample(p, host, min(args.ref_seconds, 10.0))
+    if rank == 0:
+        _, bf16_tf, peak_kind = load_peaks()
+        af = prologue_flops(p)
+        achieved = af / (kernel_ms * 1e-3) / 1e12
+        line = {
+            "metric": "TTT prologue tokens/sec on 1 B200 (1.3B layer: d_model 2048, 32 heads of 64, 32k ctx); "
+                      "% of tensor roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": p["name"], "B": B, "T": T, "H": H, "d": d, "d_model": p["d_model"],
+                       "outputs": "Q, K, V bf16 [B][H][T][d] (rotary on Q, K), eta fp32 [B][H][T]",
+                       "l2": "inputs (x 268 MB) and outputs (Q/K/V 805 MB) larger than the 126 MB L2; no flush"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16_tf, "unit": "TFLOP/s",
+                         "frac": achieved / bf16_tf, "traffic": recorded_traffic("ttt_prologue_kernel", p["name"]),
+                         "peak_kind": peak_kind, "algorithmic_flops_per_launch": af, "kernel_ms": kernel_ms,
+                         "kernel": "ttt_prologue_kernel"},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": B * T * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
+    if args.workload == PROLOGUE["name"]:
+        return run_prologue(args, world, rank, local)
     w = WORKLOADS[args.workload]
     if w.name in DECODE_WORKLOADS:
         return run_decode(args, world, rank, local)
@@ -579,7 +737,7 @@ def run_ours(args, world, rank, local):
             family = args.kernel if args.kernel != "auto" else ttt.linear_pick_impl(
                 w.B, w.H, w.T, w.d, w.mini_batch, w.dtype, w.mode)
             kname = {"tensorcore": "ttt_linear_lag_kernel", "tcgen05": "ttt_linear_umma_kernel",
-                     "tensorcore_lag2": "ttt_linear_hybrid_kernel", "generic": "ttt_linear_generic_kernel"}[family]
+                     "generic": "ttt_linear_generic_kernel"}[family]
             achieved, peak, bound, unit = ab / (kernel_ms * 1e-3) / 1e9, hbm, "hbm", "GB/s"
         traffic = recorded_traffic(kname, w.name)
         line = {
@@ -610,9 +768,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
-                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS])
-    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split", "tcgen05",
-                                             "tensorcore_lag2"],
+                    choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS]
+                    + [PROLOGUE["name"]])
+    ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split", "tcgen05"],
                     default="auto")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0,

@@ -117,11 +117,6 @@ typedef enum {
                             fp32 accumulators in tensor memory, one issuing thread), the
                             sequential per-chunk chain on warp-level mma; the state is kept
                             centred on its per-row means, which are added back to W_T, b_T */
-    TTT_IMPL_TENSORCORE_LAG2 = 5 /* TTT-Linear only, same shapes as TTT_IMPL_TENSORCORE: the state
-                                    increment on tcgen05 (fp32 in tensor memory), the products with
-                                    the state and the per-chunk chain on warp-level mma, with two
-                                    chunks of slack between the state and the chain; the state is
-                                    kept centred as in TTT_IMPL_TCGEN05 */
 } ttt_impl;
 
 /*

@@ -24,9 +24,8 @@ LIB_PATH = os.environ.get("TTT_B200_LIBRARY") or os.path.join(_PKG, "libttt_b200
 
 TTT_BF16, TTT_F32 = 0, 1
 TTT_LN_RESIDUAL, TTT_PLAIN = 0, 1
-IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3, "tcgen05": 4, "tensorcore_lag2": 5}
-_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split", 4: "tcgen05",
-               5: "tensorcore_lag2"}
+IMPLS = {"auto": 0, "generic": 1, "tensorcore": 2, "tensorcore_split": 3, "tcgen05": 4}
+_IMPL_NAMES = {0: "none", 1: "generic", 2: "tensorcore", 3: "tensorcore_split", 4: "tcgen05"}
 STATUS = ["TTT_OK", "TTT_ERR_NULL", "TTT_ERR_SHAPE", "TTT_ERR_DTYPE", "TTT_ERR_ALIGN",
           "TTT_ERR_ALIAS", "TTT_ERR_UNSUPPORTED", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT", "TTT_ERR_WORKSPACE"]
 

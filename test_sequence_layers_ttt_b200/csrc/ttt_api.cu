@@ -51,7 +51,6 @@ bool prepare() {
     return ttt::read_and_clear_device_error(&stale) == cudaSuccess &&
            ttt::read_and_clear_mlp_error(&stale) == cudaSuccess &&
            ttt::read_and_clear_umma_error(&stale) == cudaSuccess &&
-           ttt::read_and_clear_hybrid_error(&stale) == cudaSuccess &&
            ttt::read_and_clear_prologue_error(&stale) == cudaSuccess;
 }
 
@@ -75,13 +74,12 @@ ttt_status finish(cudaError_t launch, cudaStream_t stream) {
     if (launch != cudaSuccess) return TTT_ERR_CUDA;
     if (!check_env()) return TTT_OK;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
-    unsigned int flag = 0, mlp_flag = 0, umma_flag = 0, hyb_flag = 0, pro_flag = 0;
+    unsigned int flag = 0, mlp_flag = 0, umma_flag = 0, pro_flag = 0;
     if (ttt::read_and_clear_device_error(&flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_mlp_error(&mlp_flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_umma_error(&umma_flag) != cudaSuccess) return TTT_ERR_CUDA;
-    if (ttt::read_and_clear_hybrid_error(&hyb_flag) != cudaSuccess) return TTT_ERR_CUDA;
     if (ttt::read_and_clear_prologue_error(&pro_flag) != cudaSuccess) return TTT_ERR_CUDA;
-    return (flag | mlp_flag | umma_flag | hyb_flag | pro_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
+    return (flag | mlp_flag | umma_flag | pro_flag) ? TTT_ERR_TIMEOUT : TTT_OK;
 }
 
 ttt_status validate_linear(const LinearArgs& a) {
@@ -301,9 +299,6 @@ ttt_status ttt_linear_forward_impl(int B, int H, int T, int d, int mini_batch, t
         case TTT_IMPL_TCGEN05:
             if (!ttt::linear_umma_supports(a)) return TTT_ERR_UNSUPPORTED;
             return finish(ttt::launch_linear_umma(a, s), s);
-        case TTT_IMPL_TENSORCORE_LAG2:
-            if (!ttt::linear_hybrid_supports(a)) return TTT_ERR_UNSUPPORTED;
-            return finish(ttt::launch_linear_hybrid(a, s), s);
         default:
             return TTT_ERR_UNSUPPORTED;
     }
@@ -457,17 +452,16 @@ const char* ttt_status_string(ttt_status status) {
     }
 }
 
-int ttt_abi_version(void) { return 102; }
+int ttt_abi_version(void) { return 103; }
 
 #ifdef TTT_TIMELINE
 // Timeline builds only (not part of the ABI): copy the clock64 stamps of CTA 0
-// of the last launch of kernel `which` (0: ttt_linear_lag_kernel, 1:
-// ttt_linear_hybrid_kernel) into out[kTlRoles][kTlChunks][kTlEvents].
+// of the last launch of kernel `which` (0: ttt_linear_lag_kernel) into
+// out[kTlRoles][kTlChunks][kTlEvents].
 int ttt_debug_timeline(int which, long long* out) {
     if (!out) return TTT_ERR_NULL;
     if (cudaDeviceSynchronize() != cudaSuccess) return TTT_ERR_CUDA;
-    const cudaError_t e = which == 0 ? ttt::read_lag_timeline(out) : which == 1 ? ttt::read_hybrid_timeline(out)
-                                                                              : cudaErrorInvalidValue;
+    const cudaError_t e = which == 0 ? ttt::read_lag_timeline(out) : cudaErrorInvalidValue;
     return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 #endif

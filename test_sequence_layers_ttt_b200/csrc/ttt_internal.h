@@ -47,12 +47,6 @@ bool linear_umma_supports(const LinearArgs& a);
 cudaError_t launch_linear_umma(const LinearArgs& a, cudaStream_t stream);
 cudaError_t read_and_clear_umma_error(unsigned int* out);
 
-// Lag-2 scan: the state increment on tcgen05, the W products and the chain on mma.sync
-// (ttt_linear_hybrid.cu); same shapes as linear_tc.
-bool linear_hybrid_supports(const LinearArgs& a);
-cudaError_t launch_linear_hybrid(const LinearArgs& a, cudaStream_t stream);
-cudaError_t read_and_clear_hybrid_error(unsigned int* out);
-
 // Decode with the state in registers (d = 64); in place on W_T / b_T and Wm_T / bm_T.
 bool linear_decode_supports(const LinearArgs& a);
 cudaError_t launch_linear_decode(const LinearArgs& a, cudaStream_t stream);
@@ -103,7 +97,6 @@ cudaError_t read_and_clear_mlp_error(unsigned int* out);
 cudaError_t read_and_clear_device_error(unsigned int* out);
 #ifdef TTT_TIMELINE
 cudaError_t read_lag_timeline(long long* out);     // kTlRoles x kTlChunks x kTlEvents stamps
-cudaError_t read_hybrid_timeline(long long* out);
 #endif
 
 // Fault-injection hook: the chunk index named by TTT_DEBUG_DROP_CHUNK (read once

@@ -8,7 +8,7 @@ consecutive chunk steps of mid-sequence: the period of every role, the median
 time between the role's stamped points, and the median time from the chain's
 hand-off of chunk c to each consumer's pick-up.
 
-    python -m test_sequence_layers_ttt_b200.timeline [tensorcore|tensorcore_lag2]
+    python -m test_sequence_layers_ttt_b200.timeline [tensorcore]
 
 Needs a GPU.  The stamps perturb the kernel a little (one clock read and one
 store per point, CTA 0 only).
@@ -31,15 +31,6 @@ ROLES = {
         "PR": ["top", "stage free"],
         "PA": ["top", "stage in", "slot free", "done"],
         "PB": ["top", "stage in", "slot free", "done"],
-    }),
-    "tensorcore_lag2": (1, ["CH", "ST", "OW", "PR", "PA", "PB", "MMA"], {
-        "CH": ["top", "S1 correction", "stats barrier", "E formed", "E buffer free", "E handed off", "next R in"],
-        "ST": ["top", "P(c+2) done", "QW handed off", "E in", "R(c+2) handed off", "U in", "state split"],
-        "OW": ["top", "QW in", "E in", "correction done", "stats barrier", "stored"],
-        "PR": ["top", "stage free"],
-        "PA": ["top", "stage in", "slot free", "done"],
-        "PB": ["top", "stage in", "slot free", "done"],
-        "MMA": ["top", "E in", "U buffer free", "issued"],
     }),
 }
 N_ROLES, N_CHUNKS, N_EVENTS, FIRST = 8, 32, 8, 1024
@@ -90,18 +81,6 @@ def main(family: str = "tensorcore") -> None:
         # P_{j+1} handed off by WP iteration j (ev5, indexed j) -> CH load_inputs(j+1) done (ev7 of chunk j)
         d = ch[:, 7] - wp[:, 5]
         print(f"  P hand-off -> CH pick-up (same index): {np.median(d):.0f}")
-    else:
-        stw = buf[1].astype(np.float64)
-        mma = buf[6].astype(np.float64)
-        d = stw[:, 3] - ch[:, 5]
-        print(f"  E_c hand-off -> ST pick-up: {np.median(d):.0f}")
-        d = mma[:, 1] - ch[:, 5]
-        print(f"  E_c hand-off -> MMA pick-up: {np.median(d):.0f}")
-        d = stw[:, 5] - mma[:, 3]
-        print(f"  U_c issued -> ST has it: {np.median(d):.0f}")
-        # R_{c+2} handed off by ST iteration c (ev4) -> CH load_inputs(c+2) done (ev6 of chunk c+1)
-        d = ch[1:, 6] - stw[:-1, 4]
-        print(f"  R hand-off -> CH pick-up: {np.median(d):.0f}")
     if clk:
         print(f"  (SM clock {clk / 1e3:.0f} MHz nominal)")
 

@@ -45,7 +45,7 @@ def test_status_strings():
     for code, name in enumerate(b.STATUS):
         assert b.status_string(code).startswith(name)
     assert b.status_string(99) == "TTT_ERR_UNKNOWN"
-    assert b.lib.ttt_abi_version() == 102
+    assert b.lib.ttt_abi_version() == 103
 
 
 # Fake, 16-byte aligned, non-overlapping device addresses.  Never dereferenced:

@@ -107,7 +107,7 @@ def test_linear_bf16_reduced(ttt, seed, name, shape, impl):
 
 # the tensor-core families of TTT-Linear: warp-level mma with the state in
 # registers, and the state products on tcgen05 with TMEM accumulators
-TC_LINEAR = ["tensorcore", "tcgen05", "tensorcore_lag2"]
+TC_LINEAR = ["tensorcore", "tcgen05"]
 
 
 @pytest.mark.parametrize("impl", ["auto"] + TC_LINEAR)
