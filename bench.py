@@ -18,6 +18,7 @@ same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -320,11 +321,39 @@ def run_reference_prologue(args):
         "gpu_launches": 0}), flush=True)
 
 
+def run_reference_backward(args):
+    w = WORKLOADS[BACKWARD[args.workload]]
+    host = make_inputs(w, args.seed)
+    up = backward_upstream(w, args.seed)
+    for _ in range(args.warmup):
+        cpu_oracle_backward_sample(w, host, up, 0.5)
+    vals, r = [], None
+    t_start = time.perf_counter()
+    per_step = min(args.ref_seconds, 150.0 / max(args.steps, 1))
+    for _ in range(args.steps):
+        r = cpu_oracle_backward_sample(w, host, up, per_step)
+        vals.append(r["value"])
+    elapsed = time.perf_counter() - t_start
+    value = statistics.median(vals)
+    print(json.dumps({
+        "impl": "reference", "metric": f"TTT-Linear layer backward tokens/sec on 1 B200 ({w.name}); % of HBM roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_config(w), workload=args.workload, forward_workload=w.name),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0}), flush=True)
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
     if args.workload == PROLOGUE["name"]:
         return run_reference_prologue(args)
+    if args.workload in BACKWARD:
+        return run_reference_backward(args)
     w = WORKLOADS[args.workload]
     inp = make_inputs(w, args.seed)
     sample = cpu_oracle_decode_sample if args.workload in DECODE_WORKLOADS else cpu_oracle_sample
@@ -640,11 +669,156 @@ def run_prologue(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# The layer backward on a forward workload's shapes.
+BACKWARD = {"backward_1p3b_32k": "linear_1p3b_32k", "backward_125m_2k": "linear_125m_2k"}
+
+
+def backward_bytes(w) -> int:
+    """Algorithmic bytes of one ttt_linear_backward call: Q, K, V, eta and dZ
+    read and dQ, dK, dV, deta written once per head-token; W0, b0, dW_T, db_T
+    read and dW0, db0 written once per (batch, head); and the start state of
+    every mini-batch written once and read once (the method's checkpoints)."""
+    es = 2 if w.dtype == "bf16" else 4
+    per_tok = 3 * w.d * es + 4 + 4 * w.d + 3 * 4 * w.d + 4
+    state = (w.d * w.d + w.d) * 4
+    n_mb = -(-w.T // w.mini_batch)
+    return w.head_tokens * per_tok + w.B * w.H * (3 * state + 2 * n_mb * state)
+
+
+def backward_upstream(w, seed: int):
+    g = torch.Generator().manual_seed(1000 + seed)
+    return (torch.randn((w.B, w.H, w.T, w.d), generator=g), torch.randn((w.B, w.H, w.d, w.d), generator=g),
+            torch.randn((w.B, w.H, w.d), generator=g))
+
+
+def cpu_oracle_backward_sample(w, host, up, target_s: float):
+    """Time the float64 backward oracle (torch autograd over the token loop) on
+    the first tokens of one (batch, head) scan, as many as fit in about
+    target_s seconds; tokens/s in the workload's unit (B*T tokens cover all H
+    heads, so a single head's tokens count 1/H)."""
+    from oracle import backward as ob
+    sel = lambda t: t[:1, :1]
+    n, dt = 16, 0.0
+    while True:
+        sl = {k: (sel(host[k])[:, :, :n] if k in ("Q", "K", "V", "eta") else
+                  (host[k][:1] if k in ("gamma", "beta") else sel(host[k]))) for k in KEYS}
+        t0 = time.perf_counter()
+        ob.ttt_linear_backward(*(sl[k].double().numpy() for k in KEYS), sel(up[0])[:, :, :n].double().numpy(),
+                               w.mini_batch, w.mode, w.ln_eps, sel(up[1]).double().numpy(),
+                               sel(up[2]).double().numpy())
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or n >= w.T:
+            break
+        n = min(w.T, n * 4)
+    return {"value": n / w.H / dt, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of one (batch, head) scan, float64 autograd oracle, {dt:.2f} s; "
+                      f"tokens counted as head-tokens/H"}
+
+
+def run_backward(args, world, rank, local):
+    """Tokens/s of ttt_linear_backward (all three kernels of one call)."""
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+
+    w = WORKLOADS[BACKWARD[args.workload]]
+    dev = torch.device("cuda", local)
+    host = make_inputs(w, args.seed + rank)
+    up = backward_upstream(w, args.seed + rank)
+    g = {k: v.to(dev) for k, v in host.items()}
+    dZ, dW, db = (t.to(dev) for t in up)
+    f32 = dict(dtype=torch.float32, device=dev)
+    outs = [torch.empty((w.B, w.H, w.T, w.d), **f32) for _ in range(3)] + [
+        torch.empty((w.B, w.H, w.T), **f32), torch.empty((w.B, w.H, w.d, w.d), **f32),
+        torch.empty((w.B, w.H, w.d), **f32), torch.empty((w.H, w.d), **f32), torch.empty((w.H, w.d), **f32)]
+    need = ttt.linear_backward_workspace_size(w.B, w.H, w.T, w.d, w.mini_batch)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(src, dz, dw, dbb):
+        st = ttt.lib.ttt_linear_backward(
+            w.B, w.H, w.T, w.d, w.mini_batch, ttt._dtype_code(src["Q"]), ttt._mode_code("ln"), float(w.ln_eps),
+            *(ttt._ptr(src[k]) for k in KEYS), ttt._ptr(dz), ttt._ptr(dw), ttt._ptr(dbb),
+            *(ttt._ptr(o) for o in outs), ttt._ptr(ws), ctypes.c_size_t(need), ttt._stream_handle(dev, stream))
+        ttt._check(st)
+
+    for _ in range(args.warmup):
+        step(g, dZ, dW, db)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(g, dZ, dW, db)
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    ms_per_step = dist_max(start.elapsed_time(end), world) / args.steps
+    call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    value = w.B * w.T * world / (ms_per_step * 1e-3)
+
+    # end to end: every input from pinned host memory, every gradient back
+    host_in = {k: v.pin_memory() for k, v in host.items()}
+    up_in = [t.pin_memory() for t in up]
+    outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + sum(
+        t.numel() * t.element_size() for t in up_in)
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
+    dev_in = {k: torch.empty_like(v) for k, v in g.items()}
+    dev_up = [torch.empty_like(t) for t in (dZ, dW, db)]
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        for k in KEYS:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        for d_, h_ in zip(dev_up, up_in):
+            d_.copy_(h_, non_blocking=True)
+        step(dev_in, *dev_up)
+        for oh, o in zip(outs_host, outs):
+            oh.copy_(o, non_blocking=True)
+        stream.synchronize()
+    e2e_s = dist_max((time.perf_counter() - t0) / e2e_steps, world)
+
+    cpu_base = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_backward_sample(w, host, up, min(args.ref_seconds, 10.0))
+    if rank == 0:
+        hbm, _, peak_kind = load_peaks()
+        ab = backward_bytes(w)
+        achieved = ab / (call_ms * 1e-3) / 1e9
+        line = {
+            "metric": f"TTT-Linear layer backward tokens/sec on 1 B200 ({w.name}); % of HBM roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": dict(workload_config(w), workload=args.workload, forward_workload=w.name,
+                           workspace_bytes=need,
+                           step="one ttt_linear_backward call: states, reverse sweep, dgamma/dbeta (3 kernels)"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": ab,
+                         "kernel_ms": call_ms, "kernel": "ttt_linear_backward (3 kernels)"},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": w.B * w.T * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
     if args.workload == PROLOGUE["name"]:
         return run_prologue(args, world, rank, local)
+    if args.workload in BACKWARD:
+        return run_backward(args, world, rank, local)
     w = WORKLOADS[args.workload]
     if w.name in DECODE_WORKLOADS:
         return run_decode(args, world, rank, local)
@@ -769,7 +943,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
                     choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS]
-                    + [PROLOGUE["name"]])
+                    + [PROLOGUE["name"], *BACKWARD])
     ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split", "tcgen05"],
                     default="auto")
     ap.add_argument("--seed", type=int, default=0)

@@ -159,20 +159,16 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
     lo = pack_hi_halves(__float_as_uint(x0 - __uint_as_float(h0)), __float_as_uint(x1 - __uint_as_float(h1)));
 }
 
-// Cheaper split for operands that are re-split every chunk: hi = x truncated to
-// bf16 (the top half of its bit pattern), lo = (x - hi) rounded to the nearest
-// bf16.  x - hi is exact in fp32 and below 2^-7 |x|, so |x - hi - lo| <= 2^-15 |x|
-// with no bias (a truncated lo would always shorten |x|, and that bias adds up
-// over the thousands of state updates of a long sequence).  Five instructions
-// per pair: a byte permute, two masks, one packed fp32 subtraction and one
-// packed conversion.
-__device__ __forceinline__ void split_pair_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
-    hi = __byte_perm(b0, b1, 0x7632);
-    const uint32_t t0 = b0 & 0xffff0000u, t1 = b1 & 0xffff0000u;
+// The most precise split, also five instructions: hi = x rounded to the
+// nearest bf16 (one packed conversion for the pair), lo = (x - hi) rounded to
+// the nearest bf16.  |x - hi| <= 2^-8 |x| is exact in fp32, so
+// |x - hi - lo| <= 2^-16 |x|, unbiased.
+__device__ __forceinline__ void split_pair_rn(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x1), "f"(x0));
+    const uint32_t h0 = hi << 16, h1 = hi & 0xffff0000u;
     uint64_t d;
     asm("{\n .reg .b64 a, b;\n mov.b64 a, {%1, %2};\n mov.b64 b, {%3, %4};\n sub.rn.f32x2 %0, a, b;\n}\n"
-        : "=l"(d) : "r"(b0), "r"(b1), "r"(t0), "r"(t1));
+        : "=l"(d) : "f"(x0), "f"(x1), "r"(h0), "r"(h1));
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(__uint_as_float((uint32_t)(d >> 32))),
         "f"(__uint_as_float((uint32_t)d)));
 }

@@ -10,7 +10,7 @@
 //   Y_c      = X~_c W~_c
 //   G_c      = dl/dY_c (LayerNorm backward of ||X + LN(Y) - V||^2, per token)
 //   W~_{c+1} = W~_c - X~_c^T diag(eta_c) G_c
-//   zbar_c   = Q~_c W~_c - A_c G_c,  A_c[t,s] = eta_s (q_t . x_s + 1), s <= t
+//   zbar_c   = Q~_c W~_c + L_c E_c,  E_c = -diag(eta_c) G_c,  L_c[t,s] = q_t . x_s + 1, s <= t
 //   z_c      = q + LN(zbar_c)
 // Substituting the update once gives the lag-1 form used here:
 //   Y_c = P_c + M_c G_{c-1},  P_c = X~_c W~_{c-1},
@@ -21,19 +21,23 @@
 //
 // Warp roles (480 threads):
 //   CH  warps 0-3   the chain: warp w owns output features [16w, 16w+16);
-//                   writes G_c and -eta G_c as bf16 hi/lo tiles and keeps G_c
-//                   as B fragments in registers (8x8 transposes, movmatrix);
-//                   reads the next chunk's W-free inputs early in each chunk
+//                   keeps G_c as bf16 hi/lo B fragments in registers (8x8
+//                   transposes, movmatrix) and hands E_c = -eta G_c on as fp32
+//                   through a ring of four buffers; the consumers split it
+//                   themselves, so no tile packing sits on the chain
 //   WP  warps 4-7   the state: warp w keeps rows [16w, 16w+16) of W~^T (all
 //                   65 input columns, the last one the bias) as fp32 mma
-//                   accumulators; applies the update with G_{c-1}, then forms
-//                   P_{c+1} and Q~_c W~_c for its 16 features
-//   OW  warps 8-11  the output: zbar = Q~W~ - A G, LayerNorm, residual, store
+//                   accumulators; applies the update with E_{c-1}, splits the
+//                   state into bf16 hi/lo B fragments, forms P_{c+1} and hands
+//                   the fragments to the output warps
+//   OW  warps 8-11  the output: zbar = Q~W~ (from the state warps' fragments)
+//                   + L E, LayerNorm, residual, store
 //   PR  warp 12     TMA loads of K, V, Q (128-byte swizzled tiles) and eta
 //   PA  warp 13     per-chunk inputs of the chain: g.c', its row sums, eta
-//   PB  warp 14     M_c and A_c (16 x 16 tensor-core products, eta folded in)
+//   PB  warp 14     M_c (eta folded in) and L_c (16 x 16 tensor-core products)
 // Every product with an fp32 operand splits it into bf16 hi + lo terms
-// (relative error below 2^-15); bf16 inputs are exact; accumulation is fp32.
+// (both rounded to nearest: relative error at most 2^-16); bf16 inputs are
+// exact; accumulation is fp32.
 // The state is kept centred on its per-input-row means over the output
 // features (added back to W_T, b_T at the end), so y = x W + b has a mean near
 // zero and the one-pass LayerNorm variance does not cancel.
@@ -63,6 +67,8 @@ namespace {
 constexpr int D = 64;
 constexpr int NS = 8;            // TMA ring stages
 constexpr int NPRE = 8;          // ring of the chain's and output's W-free inputs
+constexpr int NGB = 4;           // ring of E_c hand-offs (chain -> state and output warps)
+constexpr int kEStride = D + 8;  // fp32 row stride of an E_c buffer (spreads the rows over the banks)
 constexpr int kCH = 4, kWP = 4, kOW = 4;
 constexpr int kWarpWP0 = kCH, kWarpOW0 = kCH + kWP, kWarpPR = kCH + kWP + kOW;
 constexpr int kWarpPA = kWarpPR + 1, kWarpPB = kWarpPR + 2;
@@ -77,13 +83,13 @@ struct LagSmem {
     unsigned char K[NS][TILE];
     unsigned char V[NS][TILE];
     unsigned char Q[NS][TILE];
-    unsigned char G[2][2][TILE];            // [buf][hi, lo] G_c, swizzled [tok][out] bf16
-    unsigned char E[2][2][TILE];            // [buf][hi, lo] -eta G_c, same layout
+    float Ef[NGB][kChunk][kEStride];        // [buf][tok][out] E_c = -eta G_c, fp32
     float4 pbuf[2][kCH][32][2];             // [buf][w][lane]: P_c fragments (8 floats)
-    float4 qwbuf[4][kCH][32][2];            // same for Q~_c W~_c, [c % 4]
+    uint4 wsplit[2][kWP][9][32];            // [j % 2][warp][group][lane]: W~_j hi (0-3), lo (4-7) B fragments
+                                            // and the bias row of the accumulator (8), for the output warps
     float4 gcbuf[NPRE][kCH][32][2];         // g * (x + beta - v) in chain fragment order
     uint4 mfrag[NPRE][2][32];               // [c % NPRE][hi, lo] -M_c as A fragments
-    uint4 afrag[NPRE][2][32];               // [c % NPRE][hi, lo] -A_c as A fragments
+    uint4 afrag[NPRE][2][32];               // [c % NPRE][hi, lo] L_c as A fragments
     float c0[NPRE][kChunk];                 // row sums of g * c'
     float etac[NPRE][kChunk];               // eta of the chunk, for the chain
     alignas(128) float eta[NS][32];
@@ -93,7 +99,7 @@ struct LagSmem {
     float u[D + 1];                         // per-input-row means removed from the state (row D: bias)
     uint64_t in_full[NS], in_empty[NS];
     uint64_t pre_full[NPRE], pre_empty[NPRE], p_full[2], p_empty[2];
-    uint64_t g_full[2], g_empty[2], qw_full[4], qw_empty[4];
+    uint64_t g_full[NGB], g_empty[NGB], qw_full[4], qw_empty[4];
     int abort_flag;
 };
 
@@ -123,6 +129,39 @@ __device__ __forceinline__ void arrive1(uint64_t* bar, int lane) {
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(bar);
 }
+// acc (16 tokens x 16 output features) = [16][64] token tile x W~ B fragments (hi + lo), starting
+// from the bias row br = (col 2t, col 2t+1 of n-tile 0, the same of n-tile 1)
+__device__ __forceinline__ void tile_product(uint32_t tile_addr, int lane, const uint32_t (&wh)[8][2],
+                                             const uint32_t (&wl)[8][2], float4 br, float (&acc)[2][4]) {
+    acc[0][0] = acc[0][2] = br.x;
+    acc[0][1] = acc[0][3] = br.y;
+    acc[1][0] = acc[1][2] = br.z;
+    acc[1][1] = acc[1][3] = br.w;
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int ks = 0; ks < 4; ks++) {
+        const int row = (mi & 1) * 8 + (lane & 7), chunk = 2 * ks + (mi >> 1);
+        uint32_t a0, a1, a2, a3;
+        ptx::ldsm_x4(tile_addr + swz_chunk(row, chunk), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < 2; nt++) {
+            ptx::mma_bf16(acc[nt], a0, a1, a2, a3, wh[2 * ks][nt], wh[2 * ks + 1][nt]);
+            ptx::mma_bf16(acc[nt], a0, a1, a2, a3, wl[2 * ks][nt], wl[2 * ks + 1][nt]);
+        }
+    }
+}
+// E_c (fp32 [tok][out]) at output features f0 = 16w + g and f0 + 8, as bf16 hi/lo pairs of tokens:
+// [0] (f0, tokens 2t, 2t+1), [1] (f0 + 8, 2t, 2t+1), [2] (f0, 2t+8, 2t+9), [3] (f0 + 8, 2t+8, 2t+9).
+// These are the A fragments of E^T (rows = features, k = tokens) and, reordered, the B fragments of
+// E (k = tokens, n = features) for the n-tiles at f0 and f0 + 8.
+__device__ __forceinline__ void load_e_pairs(const float (*E)[kEStride], int f0, int t, uint32_t (&hi)[4],
+                                             uint32_t (&lo)[4]) {
+    const int k0 = 2 * t;
+    ptx::split_pair_rn(E[k0][f0], E[k0 + 1][f0], hi[0], lo[0]);
+    ptx::split_pair_rn(E[k0][f0 + 8], E[k0 + 1][f0 + 8], hi[1], lo[1]);
+    ptx::split_pair_rn(E[k0 + 8][f0], E[k0 + 9][f0], hi[2], lo[2]);
+    ptx::split_pair_rn(E[k0 + 8][f0 + 8], E[k0 + 9][f0 + 8], hi[3], lo[3]);
+}
 
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -142,6 +181,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     volatile int* abort_flag = &s.abort_flag;
     const bool tl_lead = (tid & 31) == 0 && (warp == 0 || warp == kWarpWP0 || warp == kWarpOW0 || warp >= kWarpPR);
     (void)tl_lead;
+    TTT_TIMELINE_SMEM();
 
     if (tid < D) {
         s.gam[tid] = gamma[h * D + tid];
@@ -160,12 +200,14 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         for (int i = 0; i < 2; i++) {
             ptx::mbar_init(&s.p_full[i], kWP);
             ptx::mbar_init(&s.p_empty[i], kCH);
-            ptx::mbar_init(&s.g_full[i], kCH);
-            ptx::mbar_init(&s.g_empty[i], kWP + kOW);
             ptx::mbar_init(&s.qw_full[i], kWP);
             ptx::mbar_init(&s.qw_empty[i], kOW);
             ptx::mbar_init(&s.qw_full[i + 2], kWP);
             ptx::mbar_init(&s.qw_empty[i + 2], kOW);
+        }
+        for (int i = 0; i < NGB; i++) {
+            ptx::mbar_init(&s.g_full[i], kCH);
+            ptx::mbar_init(&s.g_empty[i], kWP + kOW);
         }
         ptx::fence_mbar_init();
     }
@@ -203,6 +245,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 }
             }
         }
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 3);
         return;
     }
 
@@ -248,6 +291,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             arrive1(&s.in_empty[slot], lane);
             TTT_STAMP(g_lag_timeline, tl_lead, 4, c, 3);
         }
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 4);
         return;
     }
 
@@ -263,7 +307,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             const uint32_t xs = ptx::smem_addr(s.K[slot]);
             const uint32_t qs = ptx::smem_addr(s.Q[slot]);
             const int mi = lane >> 3;
-            // 16x16 products: prod[0] = X_c X_{c-1}^T, prod[1] = Q_c X_c^T
+            // 16x16 products: pm = X_c X_{c-1}^T, pa = Q_c X_c^T
             float pm[2][4], pa[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; nt++)
@@ -291,7 +335,6 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     ptx::mma_bf16(pm[1], xa0, xa1, xa2, xa3, p2, p3);
                 }
             }
-            const float* eta_c = s.eta[slot];
             const float* eta_p = s.eta[pslot];
             float nm[2][4], na[2][4];
 #pragma unroll
@@ -300,17 +343,17 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 for (int r = 0; r < 4; r++) {
                     const int row = g + 8 * (r >> 1), col = 8 * nt + 2 * t + (r & 1);
                     nm[nt][r] = c > 0 ? -eta_p[col] * (pm[nt][r] + 1.f) : 0.f;
-                    na[nt][r] = col <= row ? -eta_c[col] * (pa[nt][r] + 1.f) : 0.f;
+                    na[nt][r] = col <= row ? pa[nt][r] + 1.f : 0.f;
                 }
             uint32_t mh[4], ml[4], ah[4], al[4];
-            ptx::split_pair(nm[0][0], nm[0][1], mh[0], ml[0]);
-            ptx::split_pair(nm[0][2], nm[0][3], mh[1], ml[1]);
-            ptx::split_pair(nm[1][0], nm[1][1], mh[2], ml[2]);
-            ptx::split_pair(nm[1][2], nm[1][3], mh[3], ml[3]);
-            ptx::split_pair(na[0][0], na[0][1], ah[0], al[0]);
-            ptx::split_pair(na[0][2], na[0][3], ah[1], al[1]);
-            ptx::split_pair(na[1][0], na[1][1], ah[2], al[2]);
-            ptx::split_pair(na[1][2], na[1][3], ah[3], al[3]);
+            ptx::split_pair_rn(nm[0][0], nm[0][1], mh[0], ml[0]);
+            ptx::split_pair_rn(nm[0][2], nm[0][3], mh[1], ml[1]);
+            ptx::split_pair_rn(nm[1][0], nm[1][1], mh[2], ml[2]);
+            ptx::split_pair_rn(nm[1][2], nm[1][3], mh[3], ml[3]);
+            ptx::split_pair_rn(na[0][0], na[0][1], ah[0], al[0]);
+            ptx::split_pair_rn(na[0][2], na[0][3], ah[1], al[1]);
+            ptx::split_pair_rn(na[1][0], na[1][1], ah[2], al[2]);
+            ptx::split_pair_rn(na[1][2], na[1][3], ah[3], al[3]);
             s.mfrag[b][0][lane] = make_uint4(mh[0], mh[1], mh[2], mh[3]);
             s.mfrag[b][1][lane] = make_uint4(ml[0], ml[1], ml[2], ml[3]);
             s.afrag[b][0][lane] = make_uint4(ah[0], ah[1], ah[2], ah[3]);
@@ -320,6 +363,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             TTT_STAMP(g_lag_timeline, tl_lead, 5, c, 3);
         }
         if (n > 0) arrive1(&s.in_empty[(n - 1) % NS], lane);
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 5);
         return;
     }
 
@@ -368,33 +412,31 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 #pragma unroll
             for (int jj = 0; jj < 8; jj++)
 #pragma unroll
-                for (int nt = 0; nt < 2; nt++) ptx::split_pair(Wt[jj][2 * nt], Wt[jj][2 * nt + 1], wh[jj][nt], wl[jj][nt]);
+                for (int nt = 0; nt < 2; nt++)
+                    ptx::split_pair_rn(Wt[jj][2 * nt], Wt[jj][2 * nt + 1], wh[jj][nt], wl[jj][nt]);
+        };
+        // the accumulator's starting value: the bias of this lane's output columns
+        auto bias_row = [&]() {
+            return make_float4(__shfl_sync(0xffffffffu, Bt[0], 4 * (2 * t)), __shfl_sync(0xffffffffu, Bt[0], 4 * (2 * t + 1)),
+                               __shfl_sync(0xffffffffu, Bt[2], 4 * (2 * t)), __shfl_sync(0xffffffffu, Bt[2], 4 * (2 * t + 1)));
         };
         // rows16 x W~[:, 16w..16w+16) for a [16][64] token tile, bias included
         auto product = [&](uint32_t tile_addr, float4 (&dst)[2]) {
             float acc[2][4];
-            const float b00 = __shfl_sync(0xffffffffu, Bt[0], 4 * (2 * t));
-            const float b01 = __shfl_sync(0xffffffffu, Bt[0], 4 * (2 * t + 1));
-            const float b10 = __shfl_sync(0xffffffffu, Bt[2], 4 * (2 * t));
-            const float b11 = __shfl_sync(0xffffffffu, Bt[2], 4 * (2 * t + 1));
-            acc[0][0] = acc[0][2] = b00;
-            acc[0][1] = acc[0][3] = b01;
-            acc[1][0] = acc[1][2] = b10;
-            acc[1][1] = acc[1][3] = b11;
-            const int mi = lane >> 3;
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++) {
-                const int row = (mi & 1) * 8 + (lane & 7), chunk = 2 * ks + (mi >> 1);
-                uint32_t a0, a1, a2, a3;
-                ptx::ldsm_x4(tile_addr + swz_chunk(row, chunk), a0, a1, a2, a3);
-#pragma unroll
-                for (int nt = 0; nt < 2; nt++) {
-                    ptx::mma_bf16(acc[nt], a0, a1, a2, a3, wh[2 * ks][nt], wh[2 * ks + 1][nt]);
-                    ptx::mma_bf16(acc[nt], a0, a1, a2, a3, wl[2 * ks][nt], wl[2 * ks + 1][nt]);
-                }
-            }
+            tile_product(tile_addr, lane, wh, wl, bias_row(), acc);
             dst[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
             dst[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+        };
+        // W~_j's fragments and bias row for the output warps (same lanes, same 16 output features)
+        auto publish = [&](uint4 (*dst)[32]) {
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                dst[q][lane] = make_uint4(wh[2 * q][0], wh[2 * q][1], wh[2 * q + 1][0], wh[2 * q + 1][1]);
+                dst[4 + q][lane] = make_uint4(wl[2 * q][0], wl[2 * q][1], wl[2 * q + 1][0], wl[2 * q + 1][1]);
+            }
+            const float4 br = bias_row();
+            dst[8][lane] = make_uint4(__float_as_uint(br.x), __float_as_uint(br.y), __float_as_uint(br.z),
+                                      __float_as_uint(br.w));
         };
 
         split_w();
@@ -405,22 +447,18 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             arrive1(&s.p_full[c], lane);
         }
         if (n > 0) {
-            product(ptx::smem_addr(s.Q[0]), s.qwbuf[0][w][lane]);
+            publish(s.wsplit[0][w]);
             arrive1(&s.qw_full[0], lane);
         }
 
         for (int j = 1; j <= n; j++) {
-            // ---- update with G_{j-1}: W~_j = W~_{j-1} - X~_{j-1}^T diag(eta_{j-1}) G_{j-1}
-            const int pb = (j - 1) & 1, pslot = (j - 1) % NS;
+            // ---- update with E_{j-1}: W~_j = W~_{j-1} + X~_{j-1}^T E_{j-1}
+            const int pb = (j - 1) % NGB, pslot = (j - 1) % NS;
             TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 0);
-            wait_use(&s.g_full[pb], (j - 1) >> 1, abort_flag);
+            wait_use(&s.g_full[pb], (j - 1) / NGB, abort_flag);
             TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 1);
-            uint32_t ah[4], al[4];  // -(eta G)^T: rows = features 16w.., k = tokens
-            {
-                const int mi = lane >> 3, row = (mi >> 1) * 8 + (lane & 7), chunk = 2 * w + (mi & 1);
-                ptx::ldsm_x4_t(ptx::smem_addr(s.E[pb][0]) + swz_chunk(row, chunk), ah[0], ah[1], ah[2], ah[3]);
-                ptx::ldsm_x4_t(ptx::smem_addr(s.E[pb][1]) + swz_chunk(row, chunk), al[0], al[1], al[2], al[3]);
-            }
+            uint32_t ah[4], al[4];  // E^T: rows = features 16w.., k = tokens
+            load_e_pairs(s.Ef[pb], 16 * w + g, t, ah, al);
             // The increment is formed in fresh accumulators and added to the state with fp32
             // adds (round to nearest): the tensor-core accumulation does not round to nearest,
             // and the state takes thousands of increments.
@@ -437,11 +475,10 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     ptx::mma_bf16(d0, al[0], al[1], al[2], al[3], b0, b1);
                     ptx::mma_bf16(d1, ah[0], ah[1], ah[2], ah[3], b2, b3);
                     ptx::mma_bf16(d1, al[0], al[1], al[2], al[3], b2, b3);
-#pragma unroll
-                    for (int r = 0; r < 4; r++) {
-                        Wt[2 * jp][r] += d0[r];
-                        Wt[2 * jp + 1][r] += d1[r];
-                    }
+                    ptx::add2(Wt[2 * jp][0], Wt[2 * jp][1], d0[0], d0[1]);
+                    ptx::add2(Wt[2 * jp][2], Wt[2 * jp][3], d0[2], d0[3]);
+                    ptx::add2(Wt[2 * jp + 1][0], Wt[2 * jp + 1][1], d1[0], d1[1]);
+                    ptx::add2(Wt[2 * jp + 1][2], Wt[2 * jp + 1][3], d1[2], d1[3]);
                 }
                 // bias column: x~ has a 1 in it for every token
                 float db[4] = {0.f, 0.f, 0.f, 0.f};
@@ -467,12 +504,12 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 arrive1(&s.p_full[nb], lane);
                 TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 5);
             }
-            // ---- Q~_j W~_j for the output warps
+            // ---- W~_j for the output warps, which form Q~_j W~_j
             {
-                const int qb = j & 3;
-                if (j >= 4) wait_use(&s.qw_empty[qb], (j >> 2) - 1, abort_flag);
+                const int qb = j & 1;
+                if (j >= 2) wait_use(&s.qw_empty[qb], (j >> 1) - 1, abort_flag);
                 TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 6);
-                product(ptx::smem_addr(s.Q[j % NS]), s.qwbuf[qb][w][lane]);
+                publish(s.wsplit[qb][w]);
                 arrive1(&s.qw_full[qb], lane);
                 TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 7);
             }
@@ -493,6 +530,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             b_T[(size_t)bh * D + 16 * w + g] = Bt[0] + s.u[D];
             b_T[(size_t)bh * D + 16 * w + 8 + g] = Bt[2] + s.u[D];
         }
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 1);
         return;
     }
 
@@ -565,8 +603,6 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 ptx::mma_bf16(y[1], ml.x, ml.y, ml.z, ml.w, gbh[2], gbh[3]);
             }
             TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 1);
-            if (c + 1 < n) load_pre(c + 1);
-            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 2);
             const float* gcc = gcv;
             const float* c0c = c0v;
 
@@ -601,7 +637,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                     for (int q = 0; q < 5; q++) s.red_ch[b][8 * rh + g][q][w] = sm[rh][q];
             }
             ptx::named_bar_sync(1, kCH * 32);
-            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 3);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 2);
 
             float G[2][2][2];  // [rh][nt][e]
 #pragma unroll
@@ -634,33 +670,31 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 #pragma unroll
                 for (int nt = 0; nt < 2; nt++) {
                     uint32_t hi, lo;
-                    ptx::split_pair(G[rh][nt][0], G[rh][nt][1], hi, lo);
+                    ptx::split_pair_rn(G[rh][nt][0], G[rh][nt][1], hi, lo);
                     gbh[2 * nt + rh] = ptx::movmatrix_t(hi);
                     gbl[2 * nt + rh] = ptx::movmatrix_t(lo);
                 }
-            // G_c and -eta G_c (hi/lo) -> shared tiles for the state and output warps
+            // E_c = -eta G_c in fp32 -> the state and output warps, which split it themselves
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 3);
+            const int gb = c % NGB;
+            if (c >= NGB) wait_use(&s.g_empty[gb], c / NGB - 1, abort_flag);
             TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 4);
-            if (c >= 2) wait_use(&s.g_empty[b], (c >> 1) - 1, abort_flag);
-            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 5);
 #pragma unroll
             for (int rh = 0; rh < 2; rh++)
 #pragma unroll
-                for (int nt = 0; nt < 2; nt++) {
-                    uint32_t hi, lo, ehi, elo;
-                    ptx::split_pair(G[rh][nt][0], G[rh][nt][1], hi, lo);
-                    ptx::split_pair(-etv[rh] * G[rh][nt][0], -etv[rh] * G[rh][nt][1], ehi, elo);
-                    const uint32_t off = swz(8 * rh + g, 16 * w + 8 * nt + 2 * t);
-                    *reinterpret_cast<uint32_t*>(s.G[b][0] + off) = hi;
-                    *reinterpret_cast<uint32_t*>(s.G[b][1] + off) = lo;
-                    *reinterpret_cast<uint32_t*>(s.E[b][0] + off) = ehi;
-                    *reinterpret_cast<uint32_t*>(s.E[b][1] + off) = elo;
-                }
-            __syncwarp();  // every lane's tile stores before the hand-off
-            if (lane == 0) ptx::mbar_arrive(&s.g_full[b]);
+                for (int nt = 0; nt < 2; nt++)
+                    *reinterpret_cast<float2*>(&s.Ef[gb][8 * rh + g][16 * w + 8 * nt + 2 * t]) =
+                        make_float2(-etv[rh] * G[rh][nt][0], -etv[rh] * G[rh][nt][1]);
+            __syncwarp();  // every lane's stores before the hand-off
+            if (lane == 0) ptx::mbar_arrive(&s.g_full[gb]);
+            TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 5);
+            // the next chunk's W-free inputs and P, off the chain's path
+            if (c + 1 < n) load_pre(c + 1);
             TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 6);
             if (c + 1 < n) load_inputs(c + 1);
             TTT_STAMP(g_lag_timeline, tl_lead, 0, c, 7);
         }
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 0);
         return;
     }
 
@@ -680,33 +714,44 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             const int b = c & 1, slot = c % NS;
             float z[2][4];
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 0);
-            wait_use(&s.qw_full[c & 3], c >> 2, abort_flag);
+            wait_use(&s.qw_full[c & 1], c >> 1, abort_flag);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 1);
             {
-                const float4 p0 = s.qwbuf[c & 3][w][lane][0], p1 = s.qwbuf[c & 3][w][lane][1];
-                z[0][0] = p0.x; z[0][1] = p0.y; z[0][2] = p0.z; z[0][3] = p0.w;
-                z[1][0] = p1.x; z[1][1] = p1.y; z[1][2] = p1.z; z[1][3] = p1.w;
+                // Q~_c W~_c from the state warps' fragments of W~_c
+                uint32_t wh[8][2], wl[8][2];
+                const uint4 (*src)[32] = s.wsplit[c & 1][w];
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const uint4 h = src[q][lane], l = src[4 + q][lane];
+                    wh[2 * q][0] = h.x; wh[2 * q][1] = h.y; wh[2 * q + 1][0] = h.z; wh[2 * q + 1][1] = h.w;
+                    wl[2 * q][0] = l.x; wl[2 * q][1] = l.y; wl[2 * q + 1][0] = l.z; wl[2 * q + 1][1] = l.w;
+                }
+                const uint4 bb = src[8][lane];
+                arrive1(&s.qw_empty[c & 1], lane);
+                wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
+                tile_product(ptx::smem_addr(s.Q[slot]), lane, wh, wl,
+                             make_float4(__uint_as_float(bb.x), __uint_as_float(bb.y), __uint_as_float(bb.z),
+                                         __uint_as_float(bb.w)), z);
             }
-            arrive1(&s.qw_empty[c & 3], lane);
             wait_use(&s.pre_full[c % NPRE], c / NPRE, abort_flag);
             const uint4 ah = s.afrag[c % NPRE][0][lane], al = s.afrag[c % NPRE][1][lane];
             arrive1(&s.pre_empty[c % NPRE], lane);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 2);
-            wait_use(&s.g_full[b], c >> 1, abort_flag);
+            const int gb = c % NGB;
+            wait_use(&s.g_full[gb], c / NGB, abort_flag);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 3);
             {
-                const int mi = lane >> 3, row = (mi & 1) * 8 + (lane & 7), chunk = 2 * w + (mi >> 1);
-                uint32_t gh0, gh1, gh2, gh3, gl0, gl1, gl2, gl3;
-                ptx::ldsm_x4_t(ptx::smem_addr(s.G[b][0]) + swz_chunk(row, chunk), gh0, gh1, gh2, gh3);
-                ptx::ldsm_x4_t(ptx::smem_addr(s.G[b][1]) + swz_chunk(row, chunk), gl0, gl1, gl2, gl3);
-                ptx::mma_bf16(z[0], ah.x, ah.y, ah.z, ah.w, gh0, gh1);
-                ptx::mma_bf16(z[1], ah.x, ah.y, ah.z, ah.w, gh2, gh3);
-                ptx::mma_bf16(z[0], ah.x, ah.y, ah.z, ah.w, gl0, gl1);
-                ptx::mma_bf16(z[1], ah.x, ah.y, ah.z, ah.w, gl2, gl3);
-                ptx::mma_bf16(z[0], al.x, al.y, al.z, al.w, gh0, gh1);
-                ptx::mma_bf16(z[1], al.x, al.y, al.z, al.w, gh2, gh3);
+                // zbar += L E: B fragments of E (k = tokens, n = features 16w + 8 nt + g)
+                uint32_t eh[4], el[4];
+                load_e_pairs(s.Ef[gb], 16 * w + g, t, eh, el);
+                ptx::mma_bf16(z[0], ah.x, ah.y, ah.z, ah.w, eh[0], eh[2]);
+                ptx::mma_bf16(z[1], ah.x, ah.y, ah.z, ah.w, eh[1], eh[3]);
+                ptx::mma_bf16(z[0], ah.x, ah.y, ah.z, ah.w, el[0], el[2]);
+                ptx::mma_bf16(z[1], ah.x, ah.y, ah.z, ah.w, el[1], el[3]);
+                ptx::mma_bf16(z[0], al.x, al.y, al.z, al.w, eh[0], eh[2]);
+                ptx::mma_bf16(z[1], al.x, al.y, al.z, al.w, eh[1], eh[3]);
             }
-            arrive1(&s.g_empty[b], lane);
+            arrive1(&s.g_empty[gb], lane);
 
             float ps[2][2];
 #pragma unroll
@@ -734,7 +779,6 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 4);
             ptx::named_bar_sync(2, kOW * 32);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 5);
-            wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 6);
 #pragma unroll
             for (int rh = 0; rh < 2; rh++) {
@@ -759,6 +803,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             arrive1(&s.in_empty[slot], lane);
             TTT_STAMP(g_lag_timeline, tl_lead, 2, c, 7);
         }
+        TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 2);
     }
 }
 

@@ -38,8 +38,7 @@
 //   PA  14    gamma * (x + beta - v) per (feature, token) and its row sums.
 //   PB  15    S1 (as mma B fragments), S2 and L (as hi/lo operand tiles).
 // Precision: every product with an fp32 operand splits it into bf16 hi + lo
-// (hi the truncated top half, lo the remainder rounded to nearest: |x - hi - lo|
-// at most 2^-15 |x|, unbiased) and drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
+// (both halves rounded to nearest: |x - hi - lo| at most 2^-16 |x|) and drops only lo*lo; bf16 inputs are exact; the state update is formed in TMEM
 // and added to the fp32 registers with fp32 adds (tensor-core accumulation of
 // thousands of increments would not round to nearest).
 // Feature order: accumulator row r = 16 j + i holds output feature
@@ -338,10 +337,10 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             {
                 uint32_t hi[4], lo[4];
                 // b0(nt) = S1[8nt+g][2t4, 2t4+1], b1(nt) = S1[8nt+g][2t4+8, 2t4+9]
-                ptx::split_pair(p1[0][0] + 1.f, p1[0][1] + 1.f, hi[0], lo[0]);
-                ptx::split_pair(p1[1][0] + 1.f, p1[1][1] + 1.f, hi[1], lo[1]);
-                ptx::split_pair(p1[0][2] + 1.f, p1[0][3] + 1.f, hi[2], lo[2]);
-                ptx::split_pair(p1[1][2] + 1.f, p1[1][3] + 1.f, hi[3], lo[3]);
+                ptx::split_pair_rn(p1[0][0] + 1.f, p1[0][1] + 1.f, hi[0], lo[0]);
+                ptx::split_pair_rn(p1[1][0] + 1.f, p1[1][1] + 1.f, hi[1], lo[1]);
+                ptx::split_pair_rn(p1[0][2] + 1.f, p1[0][3] + 1.f, hi[2], lo[2]);
+                ptx::split_pair_rn(p1[1][2] + 1.f, p1[1][3] + 1.f, hi[3], lo[3]);
                 ps.s1[0][lane] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 ps.s1[1][lane] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
@@ -353,12 +352,12 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                     const int t = g + 8 * rh, s0 = 8 * nt + 2 * t4;
                     const uint32_t off = tc05::kmajor16_offset(t, s0);
                     uint32_t hi, lo;
-                    ptx::split_pair(p2[nt][2 * rh] + 1.f, p2[nt][2 * rh + 1] + 1.f, hi, lo);
+                    ptx::split_pair_rn(p2[nt][2 * rh] + 1.f, p2[nt][2 * rh + 1] + 1.f, hi, lo);
                     *reinterpret_cast<uint32_t*>(ps.s2[0] + off) = hi;
                     *reinterpret_cast<uint32_t*>(ps.s2[1] + off) = lo;
                     const float l0 = s0 <= t ? pl[nt][2 * rh] + 1.f : 0.f;
                     const float l1 = s0 + 1 <= t ? pl[nt][2 * rh + 1] + 1.f : 0.f;
-                    ptx::split_pair(l0, l1, hi, lo);
+                    ptx::split_pair_rn(l0, l1, hi, lo);
                     *reinterpret_cast<uint32_t*>(ps.l[0] + off) = hi;
                     *reinterpret_cast<uint32_t*>(ps.l[1] + off) = lo;
                 }
@@ -540,17 +539,17 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
-                    ptx::split_pair_trunc(Wt[4 * j + 0], Wt[4 * j + 1], hi[2 * j], lo[2 * j]);
-                    ptx::split_pair_trunc(Wt[4 * j + 2], Wt[4 * j + 3], hi[2 * j + 1], lo[2 * j + 1]);
+                    ptx::split_pair_rn(Wt[4 * j + 0], Wt[4 * j + 1], hi[2 * j], lo[2 * j]);
+                    ptx::split_pair_rn(Wt[4 * j + 2], Wt[4 * j + 3], hi[2 * j + 1], lo[2 * j + 1]);
                 }
                 tc05::st_16x128b_x8(tq + kColWA, hi);
                 tc05::st_16x128b_x8(tq + kColWA + 32, lo);
                 uint32_t bb0 = 0u, bb1 = 0u;  // bias row: k = 0 holds b hi, k = 1 holds b lo
                 if (t4 == 0) {
                     uint32_t h, l;
-                    ptx::split_pair(bt0, 0.f, h, l);
+                    ptx::split_pair_rn(bt0, 0.f, h, l);
                     bb0 = (h & 0xffffu) | (l << 16);
-                    ptx::split_pair(bt1, 0.f, h, l);
+                    ptx::split_pair_rn(bt1, 0.f, h, l);
                     bb1 = (h & 0xffffu) | (l << 16);
                 }
                 tc05::st_16x128b_x1(tq + kColWB, bb0, bb1);
@@ -560,8 +559,8 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 uint32_t h0, l0, h1, l1;
-                ptx::split_pair(Wt[4 * j + 0], Wt[4 * j + 1], h0, l0);
-                ptx::split_pair(Wt[4 * j + 2], Wt[4 * j + 3], h1, l1);
+                ptx::split_pair_rn(Wt[4 * j + 0], Wt[4 * j + 1], h0, l0);
+                ptx::split_pair_rn(Wt[4 * j + 2], Wt[4 * j + 3], h1, l1);
                 const int k = 8 * j + 2 * t4;
                 *reinterpret_cast<uint32_t*>(s.Whi + swz(r0, k)) = h0;
                 *reinterpret_cast<uint32_t*>(s.Wlo + swz(r0, k)) = l0;
@@ -570,9 +569,9 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             }
             if (t4 == 0) {  // bias row: k = 0 holds b hi, k = 1 holds b lo
                 uint32_t h, l;
-                ptx::split_pair(bt0, 0.f, h, l);
+                ptx::split_pair_rn(bt0, 0.f, h, l);
                 *reinterpret_cast<uint32_t*>(s.Abias + tc05::kmajor16_offset(r0, 0)) = (h & 0xffffu) | (l << 16);
-                ptx::split_pair(bt1, 0.f, h, l);
+                ptx::split_pair_rn(bt1, 0.f, h, l);
                 *reinterpret_cast<uint32_t*>(s.Abias + tc05::kmajor16_offset(r1, 0)) = (h & 0xffffu) | (l << 16);
             }
             ptx::fence_proxy_async_smem();
@@ -753,10 +752,10 @@ ttt_linear_umma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                     E[nt][2 + e] = fmaf(cf.y, gc[4 * nt + 2 + e], fmaf(fmaf(cf.z, ga1, cf.w), m1, d2));
                 }
             // E_c as A fragments (rows r0/r1, k = tokens) and as hi/lo operand tiles
-            ptx::split_pair_trunc(E[0][0], E[0][1], ah[0], al[0]);
-            ptx::split_pair_trunc(E[0][2], E[0][3], ah[1], al[1]);
-            ptx::split_pair_trunc(E[1][0], E[1][1], ah[2], al[2]);
-            ptx::split_pair_trunc(E[1][2], E[1][3], ah[3], al[3]);
+            ptx::split_pair_rn(E[0][0], E[0][1], ah[0], al[0]);
+            ptx::split_pair_rn(E[0][2], E[0][3], ah[1], al[1]);
+            ptx::split_pair_rn(E[1][0], E[1][1], ah[2], al[2]);
+            ptx::split_pair_rn(E[1][2], E[1][3], ah[3], al[3]);
             const int eb = c % NE;
             if (c >= NE) wait_k(&s.e_empty[eb], c / NE - 1, abort_flag);
             if constexpr (kAInTmem) {

@@ -23,11 +23,12 @@ import numpy as np
 
 ROLES = {
     "tensorcore": (0, ["CH", "WP", "OW", "PR", "PA", "PB"], {
-        "CH": ["top", "chain mma", "next inputs", "stats barrier", "G formed", "G buffer free", "G handed off",
+        "CH": ["top", "chain mma", "stats barrier", "G formed", "E buffer free", "E handed off", "next inputs",
                "next P in"],
-        "WP": ["top", "G in", "update done", "split done", "P slot free", "P handed off", "QW slot free",
-               "QW handed off"],
-        "OW": ["top", "QW in", "A frags in", "G in", "correction done", "stats barrier", "Q tile in", "stored"],
+        "WP": ["top", "E in", "update done", "split done", "P slot free", "P handed off", "W slot free",
+               "W handed off"],
+        "OW": ["top", "W in", "QW formed + L frags in", "E in", "correction done", "stats barrier", "-",
+               "stored"],
         "PR": ["top", "stage free"],
         "PA": ["top", "stage in", "slot free", "done"],
         "PB": ["top", "stage in", "slot free", "done"],
@@ -75,9 +76,9 @@ def main(family: str = "tensorcore") -> None:
     ch = buf[0].astype(np.float64)
     if family == "tensorcore":
         wp = buf[1].astype(np.float64)
-        # G_c handed off (CH ev6 of c) -> picked up by WP iteration j = c + 1 (ev1, indexed j)
-        d = wp[1:, 1] - ch[:-1, 6]
-        print(f"  G_c hand-off -> WP pick-up: {np.median(d):.0f}")
+        # E_c handed off (CH ev5 of c) -> picked up by WP iteration j = c + 1 (ev1, indexed j)
+        d = wp[1:, 1] - ch[:-1, 5]
+        print(f"  E_c hand-off -> WP pick-up: {np.median(d):.0f}")
         # P_{j+1} handed off by WP iteration j (ev5, indexed j) -> CH load_inputs(j+1) done (ev7 of chunk j)
         d = ch[:, 7] - wp[:, 5]
         print(f"  P hand-off -> CH pick-up (same index): {np.median(d):.0f}")

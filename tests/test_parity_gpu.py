@@ -304,6 +304,25 @@ def test_linear_host_buffers_end_to_end(ttt):
     np.testing.assert_array_equal(Wh.numpy(), Wd)
 
 
+def test_linear_host_buffers_on_an_explicit_stream(ttt):
+    """CPU tensors with a caller stream: the copies in, the scan and the copies
+    back are all ordered on that stream, so the results equal the device call
+    even while other work is queued on the default stream."""
+    w = WORKLOADS["linear_125m_2k"].with_shape(B=2, H=3, T=256)
+    inp = make_inputs(w, 9)
+    side = torch.cuda.Stream()
+    busy = torch.randn(4096, 4096, device="cuda")
+    for _ in range(8):
+        busy = busy @ busy  # keep the default stream occupied
+        busy /= busy.norm()
+    Zh, Wh, bh = ttt.ttt_linear_forward(*(inp[k] for k in LINEAR_KEYS), stream=side)
+    torch.cuda.synchronize()
+    Zd, Wd, bd = gpu_linear(ttt, w, inp)
+    np.testing.assert_array_equal(Zh.numpy(), Zd)
+    np.testing.assert_array_equal(Wh.numpy(), Wd)
+    np.testing.assert_array_equal(bh.numpy(), bd)
+
+
 @pytest.mark.parametrize("mode", ["ln", "plain"])
 def test_linear_host_pipeline_uneven_groups(ttt, mode):
     """The host path cuts the scans into groups on several streams; groups of
