@@ -45,17 +45,53 @@ constexpr int LD = kMaxD + 1;  // padded row length of every [rows][d] array
 template <typename T>
 __device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i]); }
 
-// C (=|+=) alpha * op(A) op(B), op(A)(i,k) = TA ? A[k][i] : A[i][k], op(B)(k,j) = TB ? B[j][k] : B[k][j]
+// C (=|+=) alpha * op(A) op(B), op(A)(i,k) = TA ? A[k][i] : A[i][k], op(B)(k,j) = TB ? B[j][k] : B[k][j].
+// Each thread owns a TM x TN block of C in registers, so every element it loads from shared memory
+// feeds TN (or TM) multiply-adds; M % TM == 0 and N % TN == 0.
+template <bool TA, bool TB, int TM, int TN>
+__device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+                          float alpha, bool accumulate) {
+    const int tn = N / TN, tiles = (M / TM) * tn;
+    for (int tix = threadIdx.x; tix < tiles; tix += blockDim.x) {
+        const int i0 = (tix / tn) * TM, j0 = (tix % tn) * TN;
+        float acc[TM][TN];
+#pragma unroll
+        for (int ii = 0; ii < TM; ii++)
+#pragma unroll
+            for (int jj = 0; jj < TN; jj++) acc[ii][jj] = 0.f;
+        for (int k = 0; k < K; k++) {
+            float a[TM], b[TN];
+#pragma unroll
+            for (int ii = 0; ii < TM; ii++) a[ii] = TA ? A[k * lda + i0 + ii] : A[(i0 + ii) * lda + k];
+#pragma unroll
+            for (int jj = 0; jj < TN; jj++) b[jj] = TB ? B[(j0 + jj) * ldb + k] : B[k * ldb + j0 + jj];
+#pragma unroll
+            for (int ii = 0; ii < TM; ii++)
+#pragma unroll
+                for (int jj = 0; jj < TN; jj++) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
+        }
+#pragma unroll
+        for (int ii = 0; ii < TM; ii++)
+#pragma unroll
+            for (int jj = 0; jj < TN; jj++) {
+                float* c = C + (i0 + ii) * ldc + j0 + jj;
+                *c = accumulate ? fmaf(alpha, acc[ii][jj], *c) : alpha * acc[ii][jj];
+            }
+    }
+}
+// the largest register block the shape allows: 4 x 4 for d x d results, 2 x 2 or 1 x 2 for rows of
+// a mini-batch (any n up to 16, d a multiple of 16)
 template <bool TA, bool TB>
 __device__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                     float alpha, bool accumulate) {
-    for (int idx = threadIdx.x; idx < M * N; idx += blockDim.x) {
-        const int i = idx / N, j = idx % N;
-        float acc = 0.f;
-        for (int k = 0; k < K; k++)
-            acc = fmaf(TA ? A[k * lda + i] : A[i * lda + k], TB ? B[j * ldb + k] : B[k * ldb + j], acc);
-        C[i * ldc + j] = accumulate ? fmaf(alpha, acc, C[i * ldc + j]) : alpha * acc;
-    }
+    if (M % 4 == 0 && N % 4 == 0 && M * N >= 16 * (int)blockDim.x)
+        bmm_tiled<TA, TB, 4, 4>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (M % 2 == 0 && N % 2 == 0)
+        bmm_tiled<TA, TB, 2, 2>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (N % 2 == 0)
+        bmm_tiled<TA, TB, 1, 2>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else
+        bmm_tiled<TA, TB, 1, 1>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
 }
 
 struct BwdSmem {
