@@ -64,8 +64,40 @@ ttt_mlp_decode_kernel(int H, int T, int mb, int pos0, float eps, const Tin* __re
     float* W1mbh = W1_mb + bh * D * HID;
     float* W2mbh = W2_mb + bh * HID * D;
 
-    // ---- running state into registers; start state into shared memory when the call
-    // begins inside a mini-batch
+    // ---- start state into shared memory when the call begins inside a mini-batch (first,
+    // while the registers that will hold the running state are still free); running state
+    // into registers
+    if (pos0 > 0) {
+        // 128 KB of start state from L2: 16-byte loads, kBatch per matrix in flight per thread before
+        // the stores that consume them (a load-then-store loop would wait out one L2 round trip per
+        // element)
+        const float4* w1g = reinterpret_cast<const float4*>(W1mbh);
+        const float4* w2g = reinterpret_cast<const float4*>(W2mbh);
+        float4* w1s = reinterpret_cast<float4*>(s.W1s);
+        constexpr int kVec = D * HID / 4 / kThreads;  // 8 float4 per thread and matrix
+        constexpr int kBatch = 8;
+#pragma unroll
+        for (int u0 = 0; u0 < kVec; u0 += kBatch) {
+            float4 a[kBatch], c[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                a[u] = w1g[tid + (u0 + u) * kThreads];
+                c[u] = w2g[tid + (u0 + u) * kThreads];
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                w1s[tid + (u0 + u) * kThreads] = a[u];
+                const int i = 4 * (tid + (u0 + u) * kThreads);  // element of W2 [hid][out]; i % D <= D - 4
+                float* dst = s.W2s + (i / D) * LDW2 + i % D;
+                dst[0] = c[u].x;
+                dst[1] = c[u].y;
+                dst[2] = c[u].z;
+                dst[3] = c[u].w;
+            }
+        }
+        if (tid < HID) s.b1s[tid] = b1_mb[bh * HID + tid];
+        if (tid < D) s.b2s[tid] = b2_mb[bh * D + tid];
+    }
     float w1[R1], w2[R2];
 #pragma unroll
     for (int r = 0; r < R1; r++) w1[r] = W1bh[(R1 * r1 + r) * HID + k1];
@@ -76,12 +108,6 @@ ttt_mlp_decode_kernel(int H, int T, int mb, int pos0, float eps, const Tin* __re
     if (warp == 0) {
         b2r[0] = b2[bh * D + lane];
         b2r[1] = b2[bh * D + lane + 32];
-    }
-    if (pos0 > 0) {
-        for (int i = tid; i < D * HID; i += kThreads) s.W1s[i] = W1mbh[i];
-        for (int i = tid; i < HID * D; i += kThreads) s.W2s[(i / D) * LDW2 + i % D] = W2mbh[i];
-        for (int i = tid; i < HID; i += kThreads) s.b1s[i] = b1_mb[bh * HID + i];
-        if (tid < D) s.b2s[tid] = b2_mb[bh * D + tid];
     }
     if (tid < D) {
         s.gam[tid] = gamma[(long)h * D + tid];
@@ -240,9 +266,18 @@ ttt_mlp_decode_kernel(int H, int T, int mb, int pos0, float eps, const Tin* __re
         }
     } else if (restarted) {
         __syncthreads();
-        for (int i = tid; i < D * HID; i += kThreads) W1mbh[i] = s.W1s[i];
-        for (int i = tid; i < HID * D; i += kThreads) W2mbh[i] = s.W2s[(i / D) * LDW2 + i % D];
-        for (int i = tid; i < HID; i += kThreads) b1_mb[bh * HID + i] = s.b1s[i];
+        float4* w1g = reinterpret_cast<float4*>(W1mbh);
+        float4* w2g = reinterpret_cast<float4*>(W2mbh);
+        const float4* w1s = reinterpret_cast<const float4*>(s.W1s);
+        constexpr int kVec = D * HID / 4 / kThreads;
+#pragma unroll
+        for (int u = 0; u < kVec; u++) {
+            w1g[tid + u * kThreads] = w1s[tid + u * kThreads];
+            const int i = 4 * (tid + u * kThreads);
+            const float* src = s.W2s + (i / D) * LDW2 + i % D;
+            w2g[tid + u * kThreads] = make_float4(src[0], src[1], src[2], src[3]);
+        }
+        if (tid < HID) b1_mb[bh * HID + tid] = s.b1s[tid];
         if (tid < D) b2_mb[bh * D + tid] = s.b2s[tid];
     }
 }
