@@ -176,18 +176,65 @@ __device__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
     __syncthreads();
 }
 
-template <typename T>
-__device__ void load_tokens(BwdSmem& m, const T* Q, const T* K, const T* V, const float* eta, size_t base, int n,
-                            int d) {
-    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-        const int t = i / d, j = i % d;
-        const size_t gi = base * d + i;
-        m.X[t * LD + j] = ldv(K, gi);
-        m.Qm[t * LD + j] = ldv(Q, gi);
-        m.Vm[t * LD + j] = ldv(V, gi);
+// The next mini-batch's inputs, held in registers while the current one computes, so that their
+// global loads overlap the math instead of each waiting out a memory round trip.  Thread tid holds
+// elements tid + k * kBwdThreads of each array (n <= 16 tokens, d <= 64).
+template <typename T, bool kTokens, bool kBackward>
+struct Prefetch {
+    static constexpr int kTok = kMaxN * kMaxD / kBwdThreads;  // 4
+    static constexpr int kSt = kMaxD * kMaxD / kBwdThreads;   // 16
+    float x[kTok], q[kTok], v[kTok], dz[kTok], e, w[kSt], bb;
+    int n = 0;
+
+    __device__ void issue(const T* Q, const T* K, const T* V, const float* eta, const float* dZ, const float* st,
+                          size_t base, int n_, int d) {
+        n = n_;
+        const int tid = threadIdx.x;
+#pragma unroll
+        for (int k = 0; k < kTok; k++) {
+            const int i = tid + k * kBwdThreads;
+            if (i < n * d) {
+                const size_t gi = base * d + i;
+                x[k] = ldv(K, gi);
+                q[k] = ldv(Q, gi);
+                v[k] = ldv(V, gi);
+                if (kBackward) dz[k] = dZ[gi];
+            }
+        }
+        if (tid < n) e = eta[base + tid];
+        if (kBackward) {
+#pragma unroll
+            for (int k = 0; k < kSt; k++) {
+                const int i = tid + k * kBwdThreads;
+                if (i < d * d) w[k] = st[i];
+            }
+            if (tid < d) bb = st[d * d + tid];
+        }
     }
-    for (int t = threadIdx.x; t < n; t += blockDim.x) m.e[t] = eta[base + t];
-}
+    __device__ void commit(BwdSmem& m, int d) const {
+        const int tid = threadIdx.x;
+#pragma unroll
+        for (int k = 0; k < kTok; k++) {
+            const int i = tid + k * kBwdThreads;
+            if (i < n * d) {
+                const int o = (i / d) * LD + i % d;
+                m.X[o] = x[k];
+                m.Qm[o] = q[k];
+                m.Vm[o] = v[k];
+                if (kBackward) m.dZ[o] = dz[k];
+            }
+        }
+        if (tid < n) m.e[tid] = e;
+        if (kBackward) {
+#pragma unroll
+            for (int k = 0; k < kSt; k++) {
+                const int i = tid + k * kBwdThreads;
+                if (i < d * d) m.W[(i / d) * LD + i % d] = w[k];
+            }
+            if (tid < d) m.b[tid] = bb;
+        }
+    }
+};
 
 // ------------------------------------------------------------------ pass 1: states
 template <typename T>
@@ -207,12 +254,16 @@ ttt_linear_states_kernel(int T_, int d, int mb, float eps, const T* Q, const T* 
         m.bet[j] = beta[h * d + j];
     }
     __syncthreads();
+    Prefetch<T, true, false> pf;
+    if (nmb > 0) pf.issue(Q, K, V, eta, nullptr, nullptr, (size_t)bh * T_, min(mb, T_), d);
     for (int jb = 0; jb < nmb; jb++) {
         const int t0 = jb * mb, n = min(mb, T_ - t0);
         float* st = states + ((size_t)bh * nmb + jb) * sz;
         for (int i = threadIdx.x; i < d * d; i += blockDim.x) st[i] = m.W[(i / d) * LD + i % d];
         for (int j = threadIdx.x; j < d; j += blockDim.x) st[d * d + j] = m.b[j];
-        load_tokens(m, Q, K, V, eta, (size_t)bh * T_ + t0, n, d);
+        pf.commit(m, d);
+        if (jb + 1 < nmb)
+            pf.issue(Q, K, V, eta, nullptr, nullptr, (size_t)bh * T_ + t0 + mb, min(mb, T_ - t0 - mb), d);
         __syncthreads();
         chunk_inner_grad(m, n, d, eps);
         // W -= X^T diag(e) G, b -= G^T e
@@ -254,14 +305,18 @@ ttt_linear_backward_kernel(int T_, int d, int mb, float eps, const T* Q, const T
         m.dbet[j] = 0.f;
     }
     __syncthreads();
+    Prefetch<T, true, true> pf;
+    auto issue = [&](int jb) {
+        const int t0 = jb * mb;
+        pf.issue(Q, K, V, eta, dZ, states + ((size_t)bh * nmb + jb) * sz, (size_t)bh * T_ + t0, min(mb, T_ - t0),
+                 d);
+    };
+    if (nmb > 0) issue(nmb - 1);
     for (int jb = nmb - 1; jb >= 0; jb--) {
         const int t0 = jb * mb, n = min(mb, T_ - t0);
         const size_t base = (size_t)bh * T_ + t0;
-        const float* st = states + ((size_t)bh * nmb + jb) * sz;
-        for (int i = threadIdx.x; i < d * d; i += blockDim.x) m.W[(i / d) * LD + i % d] = st[i];
-        for (int j = threadIdx.x; j < d; j += blockDim.x) m.b[j] = st[d * d + j];
-        load_tokens(m, Q, K, V, eta, base, n, d);
-        for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.dZ[(i / d) * LD + i % d] = dZ[base * d + i];
+        pf.commit(m, d);
+        if (jb > 0) issue(jb - 1);
         __syncthreads();
         // ---- recompute the mini-batch's forward
         chunk_inner_grad(m, n, d, eps);
