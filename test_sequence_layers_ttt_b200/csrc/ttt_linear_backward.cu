@@ -48,9 +48,11 @@ __device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i])
 // C (=|+=) alpha * op(A) op(B), op(A)(i,k) = TA ? A[k][i] : A[i][k], op(B)(k,j) = TB ? B[j][k] : B[k][j].
 // Each thread owns a TM x TN block of C in registers, so every element it loads from shared memory
 // feeds TN (or TM) multiply-adds; M % TM == 0 and N % TN == 0.
-template <bool TA, bool TB, int TM, int TN>
-__device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+// KC > 0 fixes K at compile time (the k loop unrolls and its addressing folds into offsets).
+template <bool TA, bool TB, int TM, int TN, int KC>
+__device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K_,
                           float alpha, bool accumulate) {
+    const int K = KC > 0 ? KC : K_;
     const int tn = N / TN, tiles = (M / TM) * tn;
     for (int tix = threadIdx.x; tix < tiles; tix += blockDim.x) {
         const int i0 = (tix / tn) * TM, j0 = (tix % tn) * TN;
@@ -59,6 +61,7 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
         for (int ii = 0; ii < TM; ii++)
 #pragma unroll
             for (int jj = 0; jj < TN; jj++) acc[ii][jj] = 0.f;
+#pragma unroll(KC > 0 ? 8 : 1)
         for (int k = 0; k < K; k++) {
             float a[TM], b[TN];
 #pragma unroll
@@ -81,17 +84,28 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
 }
 // the largest register block the shape allows: 4 x 4 for d x d results, 2 x 2 or 1 x 2 for rows of
 // a mini-batch (any n up to 16, d a multiple of 16)
+template <bool TA, bool TB, int KC>
+__device__ void bmm_k(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+                      float alpha, bool accumulate) {
+    if (M % 4 == 0 && N % 4 == 0 && M * N >= 16 * (int)blockDim.x)
+        bmm_tiled<TA, TB, 4, 4, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (M % 2 == 0 && N % 2 == 0)
+        bmm_tiled<TA, TB, 2, 2, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (N % 2 == 0)
+        bmm_tiled<TA, TB, 1, 2, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else
+        bmm_tiled<TA, TB, 1, 1, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+}
+// K = 64 (the head dimension of the hot shapes) and K = 16 (a full mini-batch) unrolled
 template <bool TA, bool TB>
 __device__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                     float alpha, bool accumulate) {
-    if (M % 4 == 0 && N % 4 == 0 && M * N >= 16 * (int)blockDim.x)
-        bmm_tiled<TA, TB, 4, 4>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
-    else if (M % 2 == 0 && N % 2 == 0)
-        bmm_tiled<TA, TB, 2, 2>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
-    else if (N % 2 == 0)
-        bmm_tiled<TA, TB, 1, 2>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    if (K == 64)
+        bmm_k<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (K == 16)
+        bmm_k<TA, TB, 16>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
     else
-        bmm_tiled<TA, TB, 1, 1>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+        bmm_k<TA, TB, 0>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
 }
 
 struct BwdSmem {
