@@ -38,7 +38,7 @@ static __device__ __align__(256) unsigned char g_backward_static_workspace[kBack
 
 namespace {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 512;
 constexpr int kMaxD = 64, kMaxN = 16;
 constexpr int LD = kMaxD + 1;  // padded row length of every [rows][d] array
 
@@ -82,14 +82,18 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
             }
     }
 }
-// the largest register block the shape allows: 4 x 4 for d x d results, 2 x 2 or 1 x 2 for rows of
-// a mini-batch (any n up to 16, d a multiple of 16)
+// the register block: the largest that leaves no thread without one (4 x 4 down to 1 x 2), for any
+// n up to 16 and d a multiple of 16
 template <bool TA, bool TB, int KC>
 __device__ void bmm_k(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                       float alpha, bool accumulate) {
-    if (M % 4 == 0 && N % 4 == 0 && M * N >= 16 * (int)blockDim.x)
+    // the largest block that still gives every thread one
+    const int nt = (int)blockDim.x;
+    if (M % 4 == 0 && N % 4 == 0 && M * N >= 16 * nt)
         bmm_tiled<TA, TB, 4, 4, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
-    else if (M % 2 == 0 && N % 2 == 0)
+    else if (M % 2 == 0 && N % 4 == 0 && M * N >= 8 * nt)
+        bmm_tiled<TA, TB, 2, 4, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    else if (M % 2 == 0 && N % 2 == 0 && M * N >= 4 * nt)
         bmm_tiled<TA, TB, 2, 2, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
     else if (N % 2 == 0)
         bmm_tiled<TA, TB, 1, 2, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
@@ -195,8 +199,8 @@ __device__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
 // elements tid + k * kBwdThreads of each array (n <= 16 tokens, d <= 64).
 template <typename T, bool kTokens, bool kBackward>
 struct Prefetch {
-    static constexpr int kTok = kMaxN * kMaxD / kBwdThreads;  // 4
-    static constexpr int kSt = kMaxD * kMaxD / kBwdThreads;   // 16
+    static constexpr int kTok = kMaxN * kMaxD / kBwdThreads;  // 2
+    static constexpr int kSt = kMaxD * kMaxD / kBwdThreads;   // 8
     float x[kTok], q[kTok], v[kTok], dz[kTok], e, w[kSt], bb;
     int n = 0;
 
