@@ -53,9 +53,11 @@ template <bool TA, bool TB, int TM, int TN, int KC>
 __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K_,
                           float alpha, bool accumulate) {
     const int K = KC > 0 ? KC : K_;
-    const int tn = N / TN, tiles = (M / TM) * tn;
+    // a thread's block is strided: rows i0 + ii * (M / TM), columns j0 + jj * (N / TN), so that the
+    // lanes of a warp read consecutive columns (and one or two rows) of shared memory
+    const int tm = M / TM, tn = N / TN, tiles = tm * tn;
     for (int tix = threadIdx.x; tix < tiles; tix += blockDim.x) {
-        const int i0 = (tix / tn) * TM, j0 = (tix % tn) * TN;
+        const int i0 = tix / tn, j0 = tix % tn;
         float acc[TM][TN];
 #pragma unroll
         for (int ii = 0; ii < TM; ii++)
@@ -65,9 +67,9 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
         for (int k = 0; k < K; k++) {
             float a[TM], b[TN];
 #pragma unroll
-            for (int ii = 0; ii < TM; ii++) a[ii] = TA ? A[k * lda + i0 + ii] : A[(i0 + ii) * lda + k];
+            for (int ii = 0; ii < TM; ii++) a[ii] = TA ? A[k * lda + i0 + ii * tm] : A[(i0 + ii * tm) * lda + k];
 #pragma unroll
-            for (int jj = 0; jj < TN; jj++) b[jj] = TB ? B[(j0 + jj) * ldb + k] : B[k * ldb + j0 + jj];
+            for (int jj = 0; jj < TN; jj++) b[jj] = TB ? B[(j0 + jj * tn) * ldb + k] : B[k * ldb + j0 + jj * tn];
 #pragma unroll
             for (int ii = 0; ii < TM; ii++)
 #pragma unroll
@@ -77,7 +79,7 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
         for (int ii = 0; ii < TM; ii++)
 #pragma unroll
             for (int jj = 0; jj < TN; jj++) {
-                float* c = C + (i0 + ii) * ldc + j0 + jj;
+                float* c = C + (i0 + ii * tm) * ldc + j0 + jj * tn;
                 *c = accumulate ? fmaf(alpha, acc[ii][jj], *c) : alpha * acc[ii][jj];
             }
     }
