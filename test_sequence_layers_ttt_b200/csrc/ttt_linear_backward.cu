@@ -50,7 +50,7 @@ __device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i])
 // feeds TN (or TM) multiply-adds; M % TM == 0 and N % TN == 0.
 // KC > 0 fixes K at compile time (the k loop unrolls and its addressing folds into offsets).
 template <bool TA, bool TB, int TM, int TN, int KC>
-__device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K_,
+__device__ __forceinline__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K_,
                           float alpha, bool accumulate) {
     const int K = KC > 0 ? KC : K_;
     // a thread's block is strided: rows i0 + ii * (M / TM), columns j0 + jj * (N / TN), so that the
@@ -87,7 +87,7 @@ __device__ void bmm_tiled(float* C, int ldc, const float* A, int lda, const floa
 // the register block: the largest that leaves no thread without one (4 x 4 down to 1 x 2), for any
 // n up to 16 and d a multiple of 16
 template <bool TA, bool TB, int KC>
-__device__ void bmm_k(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+__device__ __forceinline__ void bmm_k(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                       float alpha, bool accumulate) {
     // the largest block that still gives every thread one
     const int nt = (int)blockDim.x;
@@ -104,7 +104,7 @@ __device__ void bmm_k(float* C, int ldc, const float* A, int lda, const float* B
 }
 // K = 64 (the head dimension of the hot shapes) and K = 16 (a full mini-batch) unrolled
 template <bool TA, bool TB>
-__device__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
+__device__ __forceinline__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                     float alpha, bool accumulate) {
     if (K == 64)
         bmm_k<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
@@ -127,7 +127,7 @@ struct BwdSmem {
 };
 
 // x^ = (y - mean y) s, s = (var y + eps)^(-1/2), per row of y [n][d]; one warp per row
-__device__ void ln_rows(const float* y, float* xh, float* s, int n, int d, float eps) {
+__device__ __forceinline__ void ln_rows(const float* y, float* xh, float* s, int n, int d, float eps) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int t = warp; t < n; t += nw) {
         float a = 0.f;
@@ -145,7 +145,7 @@ __device__ void ln_rows(const float* y, float* xh, float* s, int n, int d, float
 }
 
 // dy = s (dx^ - mean dx^ - x^ mean(dx^ x^)) per row, in place on dxh
-__device__ void ln_back_rows(float* dxh, const float* xh, const float* s, int n, int d) {
+__device__ __forceinline__ void ln_back_rows(float* dxh, const float* xh, const float* s, int n, int d) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int t = warp; t < n; t += nw) {
         float a = 0.f, c = 0.f;
@@ -159,7 +159,7 @@ __device__ void ln_back_rows(float* dxh, const float* xh, const float* s, int n,
 }
 
 // Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G)
-__device__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
+__device__ __forceinline__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
     bmm<false, false>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
     __syncthreads();
     for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
@@ -257,13 +257,16 @@ struct Prefetch {
 };
 
 // ------------------------------------------------------------------ pass 1: states
-template <typename T>
-__global__ void __launch_bounds__(kBwdThreads)
-ttt_linear_states_kernel(int T_, int d, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
+// DT: the head dimension, fixed at compile time so that every index computation folds
+template <typename T, int DT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+ttt_linear_states_kernel(int T_, int d_arg, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
                          const float* W0, const float* b0, const float* gamma, const float* beta, int H,
                          float* states) {
     extern __shared__ float smem_f[];
     BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
+    constexpr int d = DT;
+    (void)d_arg;
     const int bh = blockIdx.x, h = bh % H;
     const int nmb = (T_ + mb - 1) / mb;
     const size_t sz = (size_t)d * d + d;
@@ -303,14 +306,16 @@ ttt_linear_states_kernel(int T_, int d, int mb, float eps, const T* Q, const T* 
 }
 
 // ------------------------------------------------------------------ pass 2: the reverse sweep
-template <typename T>
-__global__ void __launch_bounds__(kBwdThreads)
-ttt_linear_backward_kernel(int T_, int d, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
+template <typename T, int DT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, const T* K, const T* V, const float* eta,
                            const float* gamma, const float* beta, int H, const float* states, const float* dZ,
                            const float* dW_T, const float* db_T, float* dQ, float* dK, float* dV, float* deta,
                            float* dW0, float* db0, float* gb_partial) {
     extern __shared__ float smem_f[];
     BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
+    constexpr int d = DT;
+    (void)d_arg;
     const int bh = blockIdx.x, h = bh % H;
     const int nmb = (T_ + mb - 1) / mb;
     const size_t sz = (size_t)d * d + d;
@@ -545,6 +550,43 @@ size_t linear_backward_workspace_bytes(int B, int H, int T, int d, int mini_batc
     return (bh * nmb * ((size_t)d * d + d) + bh * 2 * d) * sizeof(float);
 }
 
+namespace {
+
+template <typename T, int DT>
+cudaError_t launch_dt(const LinearBwdArgs& a, float* states, float* gb, cudaStream_t stream) {
+    const LinearArgs& f = a.f;
+    const int BH = f.B * f.H;
+    const size_t smem = sizeof(BwdSmem);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ttt_linear_states_kernel<T, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(ttt_linear_backward_kernel<T, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return e;
+    auto* Q = static_cast<const T*>(f.Q);
+    auto* K = static_cast<const T*>(f.K);
+    auto* V = static_cast<const T*>(f.V);
+    if (f.T > 0)
+        ttt_linear_states_kernel<T, DT><<<BH, kBwdThreads, smem, stream>>>(
+            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.W0, f.b0, f.gamma, f.beta, f.H, states);
+    ttt_linear_backward_kernel<T, DT><<<BH, kBwdThreads, smem, stream>>>(
+        f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T, a.dQ,
+        a.dK, a.dV, a.deta, a.dW0, a.db0, gb);
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_typed(const LinearBwdArgs& a, float* states, float* gb, cudaStream_t stream) {
+    switch (a.f.d) {
+        case 16: return launch_dt<T, 16>(a, states, gb, stream);
+        case 32: return launch_dt<T, 32>(a, states, gb, stream);
+        case 64: return launch_dt<T, 64>(a, states, gb, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
 cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cudaStream_t stream) {
     if (!linear_backward_supports(a)) return cudaErrorInvalidValue;
     const LinearArgs& f = a.f;
@@ -552,43 +594,9 @@ cudaError_t launch_linear_backward(const LinearBwdArgs& a, float* workspace, cud
     const size_t nmb = ((size_t)f.T + f.mini_batch - 1) / f.mini_batch;
     float* states = workspace;
     float* gb = workspace + (size_t)BH * nmb * ((size_t)f.d * f.d + f.d);
-    const size_t smem = sizeof(BwdSmem);
-    cudaError_t e;
-    if (f.dtype == TTT_BF16) {
-        auto* Q = static_cast<const __nv_bfloat16*>(f.Q);
-        auto* K = static_cast<const __nv_bfloat16*>(f.K);
-        auto* V = static_cast<const __nv_bfloat16*>(f.V);
-        if ((e = cudaFuncSetAttribute(ttt_linear_states_kernel<__nv_bfloat16>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(ttt_linear_backward_kernel<__nv_bfloat16>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-            return e;
-        if (f.T > 0) {
-            ttt_linear_states_kernel<<<BH, kBwdThreads, smem, stream>>>(f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V,
-                                                                         f.eta, f.W0, f.b0, f.gamma, f.beta, f.H,
-                                                                         states);
-        }
-        ttt_linear_backward_kernel<<<BH, kBwdThreads, smem, stream>>>(
-            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T,
-            a.dQ, a.dK, a.dV, a.deta, a.dW0, a.db0, gb);
-    } else {
-        auto* Q = static_cast<const float*>(f.Q);
-        auto* K = static_cast<const float*>(f.K);
-        auto* V = static_cast<const float*>(f.V);
-        if ((e = cudaFuncSetAttribute(ttt_linear_states_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(ttt_linear_backward_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess)
-            return e;
-        if (f.T > 0) {
-            ttt_linear_states_kernel<<<BH, kBwdThreads, smem, stream>>>(f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V,
-                                                                         f.eta, f.W0, f.b0, f.gamma, f.beta, f.H,
-                                                                         states);
-        }
-        ttt_linear_backward_kernel<<<BH, kBwdThreads, smem, stream>>>(
-            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T,
-            a.dQ, a.dK, a.dV, a.deta, a.dW0, a.db0, gb);
-    }
+    cudaError_t e = f.dtype == TTT_BF16 ? launch_typed<__nv_bfloat16>(a, states, gb, stream)
+                                        : launch_typed<float>(a, states, gb, stream);
+    if (e != cudaSuccess) return e;
     const int hd = f.H * f.d;
     ttt_linear_dgamma_kernel<<<(hd + 255) / 256, 256, 0, stream>>>(f.B, f.H, f.d, gb, a.dgamma, a.dbeta);
     return cudaPeekAtLastError();
