@@ -96,6 +96,8 @@ KERNEL_SOURCES = {
     "ttt_mlp_decode_kernel": ("ttt_mlp_decode.cu", "common.cuh", "ttt_internal.h"),
     "ttt_prologue_kernel": ("ttt_prologue.cu", "ptx.cuh", "tcgen05.cuh", "common.cuh", "tma_host.h",
                             "ttt_internal.h"),
+    # the three kernels of one ttt_linear_backward call share one source file
+    "ttt_linear_backward": ("ttt_linear_backward.cu", "common.cuh", "ttt_internal.h"),
 }
 
 
@@ -295,7 +297,7 @@ def cpu_oracle_decode_sample(w, inp, target_s: float):
 
 
 def run_reference_prologue(args):
-    p = PROLOGUE
+    p = PROLOGUES[args.workload]
     host = prologue_inputs(args.seed, p["B"], p["T"], p["H"], p["d"], p["d_model"])
     for _ in range(args.warmup):
         cpu_oracle_prologue_sample(p, host, 0.5)
@@ -308,8 +310,7 @@ def run_reference_prologue(args):
     elapsed = time.perf_counter() - t_start
     value = statistics.median(vals)
     print(json.dumps({
-        "impl": "reference", "metric": "TTT prologue tokens/sec on 1 B200 (1.3B layer: d_model 2048, 32 heads of "
-                                       "64, 32k ctx); % of tensor roofline",
+        "impl": "reference", "metric": prologue_metric(p),
         "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -350,7 +351,7 @@ def run_reference_backward(args):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    if args.workload == PROLOGUE["name"]:
+    if args.workload in PROLOGUES:
         return run_reference_prologue(args)
     if args.workload in BACKWARD:
         return run_reference_backward(args)
@@ -544,7 +545,17 @@ def run_decode(args, world, rank, local):
 
 # The layer's prologue on the 1.3B-layer shape: x [2, 32768, 2048] bf16 against the
 # Q/K/V and learning-rate weights of 32 heads of d = 64.
-PROLOGUE = {"name": "prologue_1p3b_32k", "B": 2, "T": 32768, "H": 32, "d": 64, "d_model": 2048}
+PROLOGUES = {
+    "prologue_1p3b_32k": {"name": "prologue_1p3b_32k", "B": 2, "T": 32768, "H": 32, "d": 64, "d_model": 2048},
+    # one 16k-token sequence (a quarter of the above, still larger than L2): the case that
+    # multi-pass ncu captures of the prologue kernel run on
+    "prologue_1p3b_16k": {"name": "prologue_1p3b_16k", "B": 1, "T": 16384, "H": 32, "d": 64, "d_model": 2048},
+}
+
+
+def prologue_metric(p) -> str:
+    return (f"TTT prologue tokens/sec on 1 B200 (1.3B layer: d_model {p['d_model']}, {p['H']} heads of {p['d']}, "
+            f"{p['T'] // 1024}k ctx); % of tensor roofline")
 
 
 def prologue_inputs(seed: int, B: int, T: int, H: int, d: int, d_model: int):
@@ -586,7 +597,7 @@ def run_prologue(args, world, rank, local):
     """Forward tokens/s of ttt_prologue_forward on the 1.3B-layer shape."""
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
-    p = PROLOGUE
+    p = PROLOGUES[args.workload]
     dev = torch.device("cuda", local)
     host = prologue_inputs(args.seed + rank, p["B"], p["T"], p["H"], p["d"], p["d_model"])
     g = [t.to(dev) for t in host]
@@ -648,14 +659,14 @@ def run_prologue(args, world, rank, local):
         af = prologue_flops(p)
         achieved = af / (kernel_ms * 1e-3) / 1e12
         line = {
-            "metric": "TTT prologue tokens/sec on 1 B200 (1.3B layer: d_model 2048, 32 heads of 64, 32k ctx); "
-                      "% of tensor roofline",
+            "metric": prologue_metric(p),
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": p["name"], "B": B, "T": T, "H": H, "d": d, "d_model": p["d_model"],
                        "outputs": "Q, K, V bf16 [B][H][T][d] (rotary on Q, K), eta fp32 [B][H][T]",
-                       "l2": "inputs (x 268 MB) and outputs (Q/K/V 805 MB) larger than the 126 MB L2; no flush"},
+                       "l2": f"inputs (x {B * T * p['d_model'] * 2 / 1e6:.0f} MB) and outputs (Q/K/V "
+                             f"{3 * B * T * H * d * 2 / 1e6:.0f} MB) larger than the 126 MB L2; no flush"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16_tf, "unit": "TFLOP/s",
                          "frac": achieved / bf16_tf, "traffic": recorded_traffic("ttt_prologue_kernel", p["name"]),
                          "peak_kind": peak_kind, "algorithmic_flops_per_launch": af, "kernel_ms": kernel_ms,
@@ -801,7 +812,8 @@ def run_backward(args, world, rank, local):
                            workspace_bytes=need,
                            step="one ttt_linear_backward call: states, reverse sweep, dgamma/dbeta (3 kernels)"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": ab,
+                         "traffic": recorded_traffic("ttt_linear_backward", args.workload),
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": ab,
                          "kernel_ms": call_ms, "kernel": "ttt_linear_backward (3 kernels)"},
             "cpu_baseline": cpu_base,
             "e2e": {"value": w.B * w.T * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -815,7 +827,7 @@ def run_backward(args, world, rank, local):
 def run_ours(args, world, rank, local):
     from test_sequence_layers_ttt_b200 import _binding as ttt
 
-    if args.workload == PROLOGUE["name"]:
+    if args.workload in PROLOGUES:
         return run_prologue(args, world, rank, local)
     if args.workload in BACKWARD:
         return run_backward(args, world, rank, local)
@@ -943,7 +955,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_1p3b_32k",
                     choices=[k for k, v in WORKLOADS.items() if v.T >= 2048 or k in DECODE_WORKLOADS]
-                    + [PROLOGUE["name"], *BACKWARD])
+                    + [*PROLOGUES, *BACKWARD])
     ap.add_argument("--kernel", choices=["auto", "generic", "tensorcore", "tensorcore_split", "tcgen05"],
                     default="auto")
     ap.add_argument("--seed", type=int, default=0)
