@@ -41,6 +41,10 @@ cudaError_t launch_linear_generic(const LinearArgs& a, cudaStream_t stream);
 
 bool linear_tc_supports(const LinearArgs& a);
 cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream);
+// The same scan as the checkpoint pass of the layer backward: stores the state at the start of
+// every mini-batch (W [in][out], then b; d^2 + d floats per mini-batch and (batch, head)) into
+// `states`; writes neither Z nor the final state (a.Z, a.W_T, a.b_T unused).
+cudaError_t launch_linear_tc_checkpoints(const LinearArgs& a, float* states, cudaStream_t stream);
 
 // State products on tcgen05 / TMEM, chain on mma.sync (ttt_linear_umma.cu); same shapes as linear_tc.
 bool linear_umma_supports(const LinearArgs& a);

@@ -9,9 +9,11 @@
 // respect to Q, K, V, eta, W0, b0, gamma and beta.
 //
 // Two passes, one CTA per (batch, head), fp32 in shared memory:
-//   1. ttt_linear_states_kernel runs the forward scan mini-batch by mini-batch
-//      and records the state each mini-batch starts from, W_j (d x d) and b_j,
-//      in the caller's workspace (d^2 + d floats per mini-batch and head).
+//   1. the forward scan records the state each mini-batch starts from, W_j
+//      (d x d) and b_j, in the caller's workspace (d^2 + d floats per
+//      mini-batch and head): the tensor-core scan kernel's checkpoint variant
+//      for bf16, d = 64, mini-batch 16 and T a multiple of 16, otherwise
+//      ttt_linear_states_kernel, mini-batch by mini-batch in fp32.
 //   2. ttt_linear_backward_kernel walks the mini-batches in reverse.  For each
 //      it reloads W_j, b_j, recomputes the mini-batch's intermediates
 //        Y = X W + b,  x^ = LN0(Y),  R = X + gamma x^ + beta - V,
@@ -585,9 +587,16 @@ cudaError_t launch_dt(const LinearBwdArgs& a, float* states, float* gb, cudaStre
     auto* Q = static_cast<const T*>(f.Q);
     auto* K = static_cast<const T*>(f.K);
     auto* V = static_cast<const T*>(f.V);
-    if (f.T > 0)
-        ttt_linear_states_kernel<T, DT><<<BH, kBwdThreads, smem, stream>>>(
-            f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.W0, f.b0, f.gamma, f.beta, f.H, states);
+    if (f.T > 0) {
+        // The tensor-core forward scan writes the checkpoints where it takes the shape (bf16, d = 64,
+        // mini-batch 16, T a multiple of 16); the fp32 states pass covers every other shape.
+        if (std::is_same<T, __nv_bfloat16>::value && DT == 64 && linear_tc_supports(f)) {
+            if ((e = launch_linear_tc_checkpoints(f, states, stream)) != cudaSuccess) return e;
+        } else {
+            ttt_linear_states_kernel<T, DT><<<BH, kBwdThreads, smem, stream>>>(
+                f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.W0, f.b0, f.gamma, f.beta, f.H, states);
+        }
+    }
     ttt_linear_backward_kernel<T, DT><<<BH, kBwdThreads, smem, stream>>>(
         f.T, f.d, f.mini_batch, f.ln_eps, Q, K, V, f.eta, f.gamma, f.beta, f.H, states, a.dZ, a.dW_T, a.db_T, a.dQ,
         a.dK, a.dV, a.deta, a.dW0, a.db0, gb);

@@ -164,12 +164,16 @@ __device__ __forceinline__ void load_e_pairs(const float (*E)[kEStride], int f0,
 }
 
 
+// kCkpt: the checkpoint pass of the layer backward.  The state warps store the state at the
+// start of every chunk (W_j [in][out], then b_j, row means added back) at ckpt + (bh n + j) (d^2 + d);
+// no Z and no final state are written, and the output warps only keep the hand-off protocol.
+template <bool kCkpt>
 __global__ void __launch_bounds__(kThreads, 1)
 ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmEta,
                       int T, int H, float eps, const float* W0, const float* b0,
                       const float* __restrict__ gamma, const float* __restrict__ beta,
-                      float* __restrict__ Z, float* W_T, float* b_T, int drop_chunk) {
+                      float* __restrict__ Z, float* W_T, float* b_T, int drop_chunk, float* __restrict__ ckpt) {
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment (128-byte TMA swizzle) by offsetting the shared array itself, so every
     // access through `s` stays a shared-memory access (an integer round trip would make them generic)
@@ -439,6 +443,26 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                                       __float_as_uint(br.w));
         };
 
+        // the state with its row means added back, as W [in][out] and b
+        auto store_state = [&](float* Wd, float* bd) {
+#pragma unroll
+            for (int jj = 0; jj < 8; jj++) {
+                const int in0 = 8 * jj + 2 * t;
+                const float u0 = s.u[in0], u1 = s.u[in0 + 1];
+                Wd[in0 * D + 16 * w + g] = Wt[jj][0] + u0;
+                Wd[(in0 + 1) * D + 16 * w + g] = Wt[jj][1] + u1;
+                Wd[in0 * D + 16 * w + 8 + g] = Wt[jj][2] + u0;
+                Wd[(in0 + 1) * D + 16 * w + 8 + g] = Wt[jj][3] + u1;
+            }
+            if (t == 0) {
+                bd[16 * w + g] = Bt[0] + s.u[D];
+                bd[16 * w + 8 + g] = Bt[2] + s.u[D];
+            }
+        };
+        constexpr size_t kCkptStride = (size_t)D * D + D;
+        float* ck = kCkpt ? ckpt + (size_t)bh * n * kCkptStride : nullptr;
+        if (kCkpt && n > 0) store_state(ck, ck + D * D);
+
         split_w();
         // P_0 = X~_0 W~_0 and P_1 = X~_1 W~_0; Q~_0 W~_0
         for (int c = 0; c < 2 && c < n; c++) {
@@ -447,7 +471,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             arrive1(&s.p_full[c], lane);
         }
         if (n > 0) {
-            publish(s.wsplit[0][w]);
+            if (!kCkpt) publish(s.wsplit[0][w]);
             arrive1(&s.qw_full[0], lane);
         }
 
@@ -491,6 +515,7 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             arrive1(&s.in_empty[pslot], lane);
             TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 2);
             if (j == n) break;
+            if (kCkpt) store_state(ck + j * kCkptStride, ck + j * kCkptStride + D * D);
 
             split_w();
             TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 3);
@@ -509,27 +534,14 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 const int qb = j & 1;
                 if (j >= 2) wait_use(&s.qw_empty[qb], (j >> 1) - 1, abort_flag);
                 TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 6);
-                publish(s.wsplit[qb][w]);
+                if (!kCkpt) publish(s.wsplit[qb][w]);
                 arrive1(&s.qw_full[qb], lane);
                 TTT_STAMP(g_lag_timeline, tl_lead, 1, j, 7);
             }
         }
 
         // final state W~_n
-        float* WTb = W_T + (size_t)bh * D * D;
-#pragma unroll
-        for (int jj = 0; jj < 8; jj++) {
-            const int in0 = 8 * jj + 2 * t;
-            const float u0 = s.u[in0], u1 = s.u[in0 + 1];
-            WTb[in0 * D + 16 * w + g] = Wt[jj][0] + u0;
-            WTb[(in0 + 1) * D + 16 * w + g] = Wt[jj][1] + u1;
-            WTb[in0 * D + 16 * w + 8 + g] = Wt[jj][2] + u0;
-            WTb[(in0 + 1) * D + 16 * w + 8 + g] = Wt[jj][3] + u1;
-        }
-        if (t == 0) {
-            b_T[(size_t)bh * D + 16 * w + g] = Bt[0] + s.u[D];
-            b_T[(size_t)bh * D + 16 * w + 8 + g] = Bt[2] + s.u[D];
-        }
+        if (!kCkpt) store_state(W_T + (size_t)bh * D * D, b_T + (size_t)bh * D);
         TTT_TIMELINE_FLUSH(g_lag_timeline, tl_lead, 1);
         return;
     }
@@ -709,6 +721,21 @@ ttt_linear_lag_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                 gamv[nt][e] = s.gam[16 * w + 8 * nt + 2 * t + e];
                 betv[nt][e] = s.bet[16 * w + 8 * nt + 2 * t + e];
             }
+        if (kCkpt) {
+            // no outputs: every hand-off is still waited for and released in order
+            for (int c = 0; c < n; c++) {
+                const int slot = c % NS, gb = c % NGB;
+                wait_use(&s.qw_full[c & 1], c >> 1, abort_flag);
+                arrive1(&s.qw_empty[c & 1], lane);
+                wait_bounded(&s.in_full[slot], (c / NS) & 1, abort_flag);
+                wait_use(&s.pre_full[c % NPRE], c / NPRE, abort_flag);
+                arrive1(&s.pre_empty[c % NPRE], lane);
+                wait_use(&s.g_full[gb], c / NGB, abort_flag);
+                arrive1(&s.g_empty[gb], lane);
+                arrive1(&s.in_empty[slot], lane);
+            }
+            return;
+        }
         float* Zbh = Z + (size_t)bh * T * D;
         for (int c = 0; c < n; c++) {
             const int b = c & 1, slot = c % NS;
@@ -822,7 +849,10 @@ bool linear_tc_supports(const LinearArgs& a) {
            a.T % kChunk == 0;
 }
 
-cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream) {
+namespace {
+
+template <bool kCkpt>
+cudaError_t launch_lag(const LinearArgs& a, float* ckpt, cudaStream_t stream) {
     if (!linear_tc_supports(a)) return cudaErrorInvalidValue;
     const int BH = a.B * a.H;
     CUtensorMap mk, mv, mq, me;
@@ -830,11 +860,21 @@ cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream) {
         !make_token_tile_map(&mq, a.Q, a.T, BH) || !make_eta_row_map(&me, a.eta, a.T, BH))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(LagSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(ttt_linear_lag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(ttt_linear_lag_kernel<kCkpt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    ttt_linear_lag_kernel<<<BH, kThreads, smem, stream>>>(mk, mv, mq, me, a.T, a.H, a.ln_eps, a.W0, a.b0, a.gamma,
-                                                           a.beta, a.Z, a.W_T, a.b_T, drop_chunk_hook());
+    ttt_linear_lag_kernel<kCkpt><<<BH, kThreads, smem, stream>>>(mk, mv, mq, me, a.T, a.H, a.ln_eps, a.W0, a.b0,
+                                                                  a.gamma, a.beta, a.Z, a.W_T, a.b_T,
+                                                                  kCkpt ? -1 : drop_chunk_hook(), ckpt);
     return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_linear_tc(const LinearArgs& a, cudaStream_t stream) { return launch_lag<false>(a, nullptr, stream); }
+
+cudaError_t launch_linear_tc_checkpoints(const LinearArgs& a, float* states, cudaStream_t stream) {
+    return launch_lag<true>(a, states, stream);
 }
 
 #ifdef TTT_TIMELINE
