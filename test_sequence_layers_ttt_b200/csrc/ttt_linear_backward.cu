@@ -30,6 +30,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "ptx.cuh"
 #include "ttt_internal.h"
 
 namespace ttt {
@@ -105,11 +106,55 @@ __device__ __forceinline__ void bmm_k(float* C, int ldc, const float* A, int lda
     else
         bmm_tiled<TA, TB, 1, 1, KC>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
 }
-// K = 64 (the head dimension of the hot shapes) and K = 16 (a full mini-batch) unrolled
-template <bool TA, bool TB>
+// The same product on the tensor cores, for M % 16 == 0, N % 8 == 0, K % 16 == 0: warps take
+// the 16 x 8 tiles of C in turn; each fp32 operand element is split into bf16 hi + lo (both rounded
+// to nearest, |x - hi - lo| <= 2^-16 |x|) and a tile accumulates hi.hi + hi.lo + lo.hi over k in fp32
+// (mma.sync m16n8k16).  Fragments are read element by element from the fp32 arrays.
+template <bool TA, bool TB, int KC>
+__device__ __forceinline__ void bmm_mma(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N,
+                                        int K_, float alpha, bool accumulate) {
+    const int K = KC > 0 ? KC : K_;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int tn = N / 8, tiles = (M / 16) * tn;
+    auto a_at = [&](int i, int k) { return TA ? A[k * lda + i] : A[i * lda + k]; };
+    auto b_at = [&](int k, int j) { return TB ? B[j * ldb + k] : B[k * ldb + j]; };
+    for (int tix = warp; tix < tiles; tix += nw) {
+        const int i0 = (tix / tn) * 16, j0 = (tix % tn) * 8;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll(KC > 0 ? 4 : 1)
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            ptx::split_pair_rn(a_at(i0 + g, k0 + 2 * t), a_at(i0 + g, k0 + 2 * t + 1), ah[0], al[0]);
+            ptx::split_pair_rn(a_at(i0 + g + 8, k0 + 2 * t), a_at(i0 + g + 8, k0 + 2 * t + 1), ah[1], al[1]);
+            ptx::split_pair_rn(a_at(i0 + g, k0 + 2 * t + 8), a_at(i0 + g, k0 + 2 * t + 9), ah[2], al[2]);
+            ptx::split_pair_rn(a_at(i0 + g + 8, k0 + 2 * t + 8), a_at(i0 + g + 8, k0 + 2 * t + 9), ah[3], al[3]);
+            ptx::split_pair_rn(b_at(k0 + 2 * t, j0 + g), b_at(k0 + 2 * t + 1, j0 + g), bh[0], bl[0]);
+            ptx::split_pair_rn(b_at(k0 + 2 * t + 8, j0 + g), b_at(k0 + 2 * t + 9, j0 + g), bh[1], bl[1]);
+            ptx::mma_bf16(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+            ptx::mma_bf16(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+            ptx::mma_bf16(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            float* c = C + (i0 + g + 8 * (r >> 1)) * ldc + j0 + 2 * t + (r & 1);
+            *c = accumulate ? fmaf(alpha, acc[r], *c) : alpha * acc[r];
+        }
+    }
+}
+// K = 64 (the head dimension of the hot shapes) and K = 16 (a full mini-batch) unrolled; with kTC
+// (the d = 64 kernels) the shapes the tensor cores take go there
+template <bool TA, bool TB, bool kTC>
 __device__ __forceinline__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
                     float alpha, bool accumulate) {
-    if (K == 64)
+    if (kTC && M % 16 == 0 && N % 8 == 0 && K % 16 == 0) {
+        if (K == 64)
+            bmm_mma<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+        else if (K == 16)
+            bmm_mma<TA, TB, 16>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+        else
+            bmm_mma<TA, TB, 0>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+    } else if (K == 64)
         bmm_k<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
     else if (K == 16)
         bmm_k<TA, TB, 16>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
@@ -162,8 +207,9 @@ __device__ __forceinline__ void ln_back_rows(float* dxh, const float* xh, const 
 }
 
 // Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G)
+template <bool kTC>
 __device__ __forceinline__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
-    bmm<false, false>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
+    bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
     __syncthreads();
     for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
     __syncthreads();
@@ -269,6 +315,7 @@ ttt_linear_states_kernel(int T_, int d_arg, int mb, float eps, const T* Q, const
     extern __shared__ float smem_f[];
     BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
     constexpr int d = DT;
+    constexpr bool kTC = DT == 64;  // products on the tensor cores
     (void)d_arg;
     const int bh = blockIdx.x, h = bh % H;
     const int nmb = (T_ + mb - 1) / mb;
@@ -295,14 +342,14 @@ ttt_linear_states_kernel(int T_, int d_arg, int mb, float eps, const T* Q, const
         auto chunk = [&](auto nc) {
             constexpr int NC = decltype(nc)::value;
             const int n = NC > 0 ? NC : n_rt;
-            chunk_inner_grad(m, n, d, eps);
+            chunk_inner_grad<kTC>(m, n, d, eps);
             // W -= X^T diag(e) G, b -= G^T e
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, o = t * LD + i % d;
                 m.tmp[o] = m.e[t] * m.G[o];
             }
             __syncthreads();
-            bmm<true, false>(m.W, LD, m.X, LD, m.tmp, LD, d, d, n, -1.f, true);
+            bmm<true, false, kTC>(m.W, LD, m.X, LD, m.tmp, LD, d, d, n, -1.f, true);
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
@@ -327,6 +374,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
     extern __shared__ float smem_f[];
     BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
     constexpr int d = DT;
+    constexpr bool kTC = DT == 64;  // products on the tensor cores
     (void)d_arg;
     const int bh = blockIdx.x, h = bh % H;
     const int nmb = (T_ + mb - 1) / mb;
@@ -360,8 +408,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             constexpr int NC = decltype(nc)::value;
             const int n = NC > 0 ? NC : n_rt;
             // ---- recompute the mini-batch's forward
-            chunk_inner_grad(m, n, d, eps);
-            bmm<false, true>(m.P, kMaxN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
+            chunk_inner_grad<kTC>(m, n, d, eps);
+            bmm<false, true, kTC>(m.P, kMaxN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
             __syncthreads();
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
@@ -369,9 +417,9 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             }
             __syncthreads();
             // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb)
-            bmm<false, false>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false);
+            bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false);
             __syncthreads();
-            bmm<false, false>(m.tmp, LD, m.A, kMaxN, m.G, LD, n, d, n, -1.f, true);
+            bmm<false, false, kTC>(m.tmp, LD, m.A, kMaxN, m.G, LD, n, d, n, -1.f, true);
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
             __syncthreads();
@@ -396,10 +444,10 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             ln_back_rows(m.dZb, m.zh, m.s2, n, d);
             __syncthreads();
             // ---- Zb = Q W + b - A G
-            bmm<false, true>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true);      // dQ += dZb W^T
-            bmm<true, false>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);    // dW_prev = Q^T dZb
-            bmm<false, true>(m.dA, kMaxN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
-            bmm<true, false>(m.dG, LD, m.A, kMaxN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
+            bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true);      // dQ += dZb W^T
+            bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);    // dW_prev = Q^T dZb
+            bmm<false, true, kTC>(m.dA, kMaxN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
+            bmm<true, false, kTC>(m.dG, LD, m.A, kMaxN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.dZb[t * LD + j];
@@ -411,7 +459,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 if (s_ > t) m.dA[t * kMaxN + s_] = 0.f;
             }
             // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp)
-            bmm<false, false>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false);
+            bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false);
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
@@ -438,7 +486,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 m.tmp[o] = m.e[t] * m.G[o];
             }
             __syncthreads();
-            bmm<false, true>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false);
+            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false);
             // dW_prev += dW (the state passes through)
             for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
                 const int o = (i / d) * LD + i % d;
@@ -447,8 +495,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * kMaxN + i % n] *= m.e[i % n];
             __syncthreads();
-            bmm<false, false>(m.dQc, LD, m.dA, kMaxN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
-            bmm<true, false>(m.dXc, LD, m.dA, kMaxN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
+            bmm<false, false, kTC>(m.dQc, LD, m.dA, kMaxN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
+            bmm<true, false, kTC>(m.dXc, LD, m.dA, kMaxN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
             // ---- G = s (Gx - m1 - x^ m2), Gx = 2 gamma R, R = X + gamma x^ + beta - V
             {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -508,8 +556,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             }
             __syncthreads();
             // ---- Y = X W + b
-            bmm<false, true>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true);     // dX += dY W^T
-            bmm<true, false>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true);     // dW_prev += X^T dY
+            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true);     // dX += dY W^T
+            bmm<true, false, kTC>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true);     // dW_prev += X^T dY
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
