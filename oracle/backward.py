@@ -37,14 +37,14 @@ MODE_LN_RESIDUAL = 0
 MODE_PLAIN = 1
 
 
-def _t(x, requires_grad=False):
+def _t(x, requires_grad=False, dtype=torch.float64):
     if x is None:
         return None
     if hasattr(x, "detach"):
         t = x.detach().to("cpu", torch.float64).clone()
     else:
         t = torch.as_tensor(np.asarray(x, dtype=np.float64)).clone()
-    return t.requires_grad_(requires_grad)
+    return t.to(dtype).requires_grad_(requires_grad)
 
 
 def _inner_grad(k, v, Ws, bs, gamma, beta, mode: int, eps: float):
@@ -98,22 +98,27 @@ def linear_scan(Q, K, V, eta, W0, b0, gamma, beta, mini_batch: int, mode: int, e
 
 def ttt_linear_backward(Q, K, V, eta, W0, b0, gamma, beta, dZ, mini_batch: int,
                         mode: int = MODE_LN_RESIDUAL, ln_eps: float = 1e-6,
-                        dW_T=None, db_T=None) -> Tuple[np.ndarray, ...]:
+                        dW_T=None, db_T=None, dtype=torch.float64) -> Tuple[np.ndarray, ...]:
     """Gradients of sum(Z dZ) + sum(W_T dW_T) + sum(b_T db_T) with respect to
     (Q, K, V, eta, W0, b0, gamma, beta).  In plain mode b0, gamma, beta may be
-    None and their gradients are returned as None."""
+    None and their gradients are returned as None.
+
+    ``dtype=torch.float32`` evaluates the same steps in single precision: not a
+    reference, but the rounding floor of any fp32 implementation of the scan's
+    backward, against which a long sequence's fp32 errors are judged."""
     plain = mode == MODE_PLAIN
-    Qt, Kt, Vt, et, W0t = (_t(x, True) for x in (Q, K, V, eta, W0))
+    c = lambda x, rg=False: _t(x, rg, dtype)
+    Qt, Kt, Vt, et, W0t = (c(x, True) for x in (Q, K, V, eta, W0))
     B, H, T, d = Qt.shape
-    b0t = _t(b0 if b0 is not None else np.zeros((B, H, d)), not plain)
-    gt = _t(gamma, not plain) if not plain else None
-    bt = _t(beta, not plain) if not plain else None
+    b0t = c(b0 if b0 is not None else np.zeros((B, H, d)), not plain)
+    gt = c(gamma, not plain) if not plain else None
+    bt = c(beta, not plain) if not plain else None
     Z, W_T, b_T = linear_scan(Qt, Kt, Vt, et, W0t, b0t, gt, bt, mini_batch, mode, ln_eps)
-    L = (Z * _t(dZ)).sum()
+    L = (Z * c(dZ)).sum()
     if dW_T is not None:
-        L = L + (W_T * _t(dW_T)).sum()
+        L = L + (W_T * c(dW_T)).sum()
     if db_T is not None and not plain:
-        L = L + (b_T * _t(db_T)).sum()
+        L = L + (b_T * c(db_T)).sum()
     wrt = [Qt, Kt, Vt, et, W0t] + ([] if plain else [b0t, gt, bt])
     grads = torch.autograd.grad(L, wrt, allow_unused=True)
     out = [None if gr is None else gr.numpy() for gr in grads]

@@ -91,6 +91,36 @@ def test_linear_backward_125m_heads(ttt):
     check(ttt, w, inp, *upstream(w, 0), 16)
 
 
+# Long sequences: the gradients of the first tokens are carried back through every
+# later mini-batch, and fp32 rounding grows along that path.  The same steps as the
+# oracle, evaluated in float32 on the CPU, miss the float64 result by about 1.5e-2 of
+# RMS (dK) at 4096 tokens of the 1.3B-layer shape, so the 1e-3 bar cannot hold for any
+# fp32 implementation there.  The bar is four times that fp32 floor, per gradient, and
+# never below 1e-3.
+FLOOR_FACTOR = 4.0
+
+
+def test_linear_backward_long_sequence(ttt):
+    """One head of the 1.3B-layer shape over 4096 tokens (256 mini-batches)."""
+    w = WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=1, T=4096)
+    inp = make_inputs(w, 2)
+    dZ, dW, db = upstream(w, 2)
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    got = ttt.ttt_linear_backward(*(inp[k].cuda() for k in keys), dZ.cuda(), dW.cuda(), db.cuda(), mini_batch=16,
+                                  ln_eps=w.ln_eps)
+    torch.cuda.synchronize()
+    ref = ob.ttt_linear_backward(*(inp[k] for k in keys), dZ, 16, ln_eps=w.ln_eps, dW_T=dW, db_T=db)
+    f32 = ob.ttt_linear_backward(*(inp[k] for k in keys), dZ, 16, ln_eps=w.ln_eps, dW_T=dW, db_T=db,
+                                 dtype=torch.float32)
+    for name, a, r, f in zip(NAMES, got, ref, f32):
+        a = a.cpu().numpy().astype(np.float64)
+        assert np.isfinite(a).all(), f"{name}: non-finite"
+        floor = float(np.abs(np.asarray(f, dtype=np.float64) - r).max()) / rms(r)
+        err = float(np.abs(a - r).max()) / rms(r)
+        bar = max(BAR, FLOOR_FACTOR * floor)
+        assert err <= bar, f"{name}: max err {err:.2e} of RMS > {bar:.2e} (fp32 floor {floor:.2e})"
+
+
 def test_linear_backward_empty_sequence(ttt):
     """T = 0: dW0 = dW_T, db0 = db_T, dgamma = dbeta = 0."""
     w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=0)

@@ -81,6 +81,22 @@ def test_gradients_equal_finite_differences_of_the_c_oracle(mode, mb):
         assert rel(grads[i], fd) < 1e-6, f"d{name}: {rel(grads[i], fd):.2e}"
 
 
+def test_float32_evaluation_is_the_same_algorithm():
+    """The backward oracle's single-precision evaluation (the fp32 floor used to
+    judge long sequences) runs the same steps: on a short, well-conditioned case
+    it agrees with the float64 result to single-precision rounding, and its
+    outputs are float32."""
+    import torch
+    Q, K, V, eta, W0, b0, gamma, beta, dZ, dW, db = case(5, T=24, d=8, B=1, H=2)
+    g64 = ob.ttt_linear_backward(Q, K, V, eta, W0, b0, gamma, beta, dZ, 8, LN, dW_T=dW, db_T=db)
+    g32 = ob.ttt_linear_backward(Q, K, V, eta, W0, b0, gamma, beta, dZ, 8, LN, dW_T=dW, db_T=db,
+                                 dtype=torch.float32)
+    for a, b in zip(g32, g64):
+        assert a.dtype == np.float32
+        assert rel(a, b) < 1e-4
+        assert rel(a, b) > 0  # rounded, not a copy of the float64 result
+
+
 def test_theorem1_gradients_closed_form():
     """Plain f, eta as given, W0 = 0 and one mini-batch over all T tokens:
     z_t = sum_{s<=t} 2 eta_s (q_t . k_s) v_s, so with upstream dZ
