@@ -45,6 +45,7 @@ namespace {
 constexpr int kBwdThreads = 512;
 constexpr int kMaxD = 64, kMaxN = 16;
 constexpr int LD = kMaxD + 1;  // padded row length of every [rows][d] array
+constexpr int LDN = kMaxN + 1;  // padded row length of the [n][n] token-pair arrays
 
 template <typename T>
 __device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i]); }
@@ -119,18 +120,24 @@ __device__ __forceinline__ void bmm_mma(float* C, int ldc, const float* A, int l
     const int tn = N / 8, tiles = (M / 16) * tn;
     auto a_at = [&](int i, int k) { return TA ? A[k * lda + i] : A[i * lda + k]; };
     auto b_at = [&](int k, int j) { return TB ? B[j * ldb + k] : B[k * ldb + j]; };
+    // The sum over k may visit k in any order that A and B share.  Position m (0..15) of k-step s
+    // takes k = s + 4 m when K = 64 and k = 4 (m % 4) + m / 4 when K = 16, so that the eight row
+    // lanes g and four pair lanes t of a fragment load fall in distinct banks of the 65-float rows
+    // (bank g + 8 t + s for K = 64; at most two lanes per bank for K = 16).
+    auto kk = [&](int s, int m) { return KC == 64 ? s + 4 * m : (KC == 16 ? 4 * (m & 3) + (m >> 2) : 16 * s + m); };
     for (int tix = warp; tix < tiles; tix += nw) {
         const int i0 = (tix / tn) * 16, j0 = (tix % tn) * 8;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll(KC > 0 ? 4 : 1)
-        for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int s = 0; s < K / 16; s++) {
+            const int k0 = kk(s, 2 * t), k1 = kk(s, 2 * t + 1), k8 = kk(s, 2 * t + 8), k9 = kk(s, 2 * t + 9);
             uint32_t ah[4], al[4], bh[2], bl[2];
-            ptx::split_pair_rn(a_at(i0 + g, k0 + 2 * t), a_at(i0 + g, k0 + 2 * t + 1), ah[0], al[0]);
-            ptx::split_pair_rn(a_at(i0 + g + 8, k0 + 2 * t), a_at(i0 + g + 8, k0 + 2 * t + 1), ah[1], al[1]);
-            ptx::split_pair_rn(a_at(i0 + g, k0 + 2 * t + 8), a_at(i0 + g, k0 + 2 * t + 9), ah[2], al[2]);
-            ptx::split_pair_rn(a_at(i0 + g + 8, k0 + 2 * t + 8), a_at(i0 + g + 8, k0 + 2 * t + 9), ah[3], al[3]);
-            ptx::split_pair_rn(b_at(k0 + 2 * t, j0 + g), b_at(k0 + 2 * t + 1, j0 + g), bh[0], bl[0]);
-            ptx::split_pair_rn(b_at(k0 + 2 * t + 8, j0 + g), b_at(k0 + 2 * t + 9, j0 + g), bh[1], bl[1]);
+            ptx::split_pair_rn(a_at(i0 + g, k0), a_at(i0 + g, k1), ah[0], al[0]);
+            ptx::split_pair_rn(a_at(i0 + g + 8, k0), a_at(i0 + g + 8, k1), ah[1], al[1]);
+            ptx::split_pair_rn(a_at(i0 + g, k8), a_at(i0 + g, k9), ah[2], al[2]);
+            ptx::split_pair_rn(a_at(i0 + g + 8, k8), a_at(i0 + g + 8, k9), ah[3], al[3]);
+            ptx::split_pair_rn(b_at(k0, j0 + g), b_at(k1, j0 + g), bh[0], bl[0]);
+            ptx::split_pair_rn(b_at(k8, j0 + g), b_at(k9, j0 + g), bh[1], bl[1]);
             ptx::mma_bf16(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
             ptx::mma_bf16(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
             ptx::mma_bf16(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
@@ -169,7 +176,7 @@ struct BwdSmem {
     float X[kMaxN * LD], Qm[kMaxN * LD], Vm[kMaxN * LD], dZ[kMaxN * LD];
     float xh[kMaxN * LD], R[kMaxN * LD], Gx[kMaxN * LD], G[kMaxN * LD], zh[kMaxN * LD];
     float dZb[kMaxN * LD], dG[kMaxN * LD], dQc[kMaxN * LD], dXc[kMaxN * LD], tmp[kMaxN * LD];
-    float P[kMaxN * kMaxN], A[kMaxN * kMaxN], dA[kMaxN * kMaxN];
+    float P[kMaxN * LDN], A[kMaxN * LDN], dA[kMaxN * LDN];
     float s[kMaxN], s2[kMaxN], m1[kMaxN], m2[kMaxN], mdg[kMaxN], ds[kMaxN], e[kMaxN], de[kMaxN];
     float gam[kMaxD], bet[kMaxD], dgam[kMaxD], dbet[kMaxD];
 };
@@ -409,17 +416,17 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             const int n = NC > 0 ? NC : n_rt;
             // ---- recompute the mini-batch's forward
             chunk_inner_grad<kTC>(m, n, d, eps);
-            bmm<false, true, kTC>(m.P, kMaxN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
+            bmm<false, true, kTC>(m.P, LDN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
             __syncthreads();
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
-                m.A[t * kMaxN + s_] = s_ <= t ? m.e[s_] * (m.P[t * kMaxN + s_] + 1.f) : 0.f;
+                m.A[t * LDN + s_] = s_ <= t ? m.e[s_] * (m.P[t * LDN + s_] + 1.f) : 0.f;
             }
             __syncthreads();
             // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb)
             bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false);
             __syncthreads();
-            bmm<false, false, kTC>(m.tmp, LD, m.A, kMaxN, m.G, LD, n, d, n, -1.f, true);
+            bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true);
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
             __syncthreads();
@@ -446,8 +453,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- Zb = Q W + b - A G
             bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true);      // dQ += dZb W^T
             bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);    // dW_prev = Q^T dZb
-            bmm<false, true, kTC>(m.dA, kMaxN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
-            bmm<true, false, kTC>(m.dG, LD, m.A, kMaxN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
+            bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
+            bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.dZb[t * LD + j];
@@ -456,7 +463,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             __syncthreads();
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
-                if (s_ > t) m.dA[t * kMaxN + s_] = 0.f;
+                if (s_ > t) m.dA[t * LDN + s_] = 0.f;
             }
             // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp)
             bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false);
@@ -474,7 +481,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                     for (int j = lane; j < d; j += 32) a = fmaf(m.tmp[t * LD + j], m.G[t * LD + j], a);
                     a = warp_sum(a);
                     float c = 0.f;
-                    for (int r = lane; r < n; r += 32) c = fmaf(m.dA[r * kMaxN + t], m.P[r * kMaxN + t] + 1.f, c);
+                    for (int r = lane; r < n; r += 32) c = fmaf(m.dA[r * LDN + t], m.P[r * LDN + t] + 1.f, c);
                     c = warp_sum(c);
                     if (lane == 0) m.de[t] = a + c;
                 }
@@ -493,10 +500,10 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 m.dWp[o] += m.dW[o];
             }
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
-            for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * kMaxN + i % n] *= m.e[i % n];
+            for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
-            bmm<false, false, kTC>(m.dQc, LD, m.dA, kMaxN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
-            bmm<true, false, kTC>(m.dXc, LD, m.dA, kMaxN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
+            bmm<false, false, kTC>(m.dQc, LD, m.dA, LDN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
+            bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
             // ---- G = s (Gx - m1 - x^ m2), Gx = 2 gamma R, R = X + gamma x^ + beta - V
             {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
