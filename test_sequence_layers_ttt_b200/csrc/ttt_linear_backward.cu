@@ -113,10 +113,12 @@ __device__ __forceinline__ void bmm_k(float* C, int ldc, const float* A, int lda
 // (mma.sync m16n8k16).  Fragments are read element by element from the fp32 arrays.
 template <bool TA, bool TB, int KC>
 __device__ __forceinline__ void bmm_mma(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N,
-                                        int K_, float alpha, bool accumulate) {
+                                        int K_, float alpha, bool accumulate, int w0, int wn) {
     const int K = KC > 0 ? KC : K_;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int wr = warp - w0;  // this warp's place in the range of warps the product runs on
+    if (wr < 0 || wr >= wn) return;
     const int tn = N / 8, tiles = (M / 16) * tn;
     auto a_at = [&](int i, int k) { return TA ? A[k * lda + i] : A[i * lda + k]; };
     auto b_at = [&](int k, int j) { return TB ? B[j * ldb + k] : B[k * ldb + j]; };
@@ -125,7 +127,7 @@ __device__ __forceinline__ void bmm_mma(float* C, int ldc, const float* A, int l
     // lanes g and four pair lanes t of a fragment load fall in distinct banks of the 65-float rows
     // (bank g + 8 t + s for K = 64; at most two lanes per bank for K = 16).
     auto kk = [&](int s, int m) { return KC == 64 ? s + 4 * m : (KC == 16 ? 4 * (m & 3) + (m >> 2) : 16 * s + m); };
-    for (int tix = warp; tix < tiles; tix += nw) {
+    for (int tix = wr; tix < tiles; tix += wn) {
         const int i0 = (tix / tn) * 16, j0 = (tix % tn) * 8;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll(KC > 0 ? 4 : 1)
@@ -150,17 +152,18 @@ __device__ __forceinline__ void bmm_mma(float* C, int ldc, const float* A, int l
     }
 }
 // K = 64 (the head dimension of the hot shapes) and K = 16 (a full mini-batch) unrolled; with kTC
-// (the d = 64 kernels) the shapes the tensor cores take go there
+// (the d = 64 kernels) the shapes the tensor cores take go there, on warps [w0, w0 + wn) only, so
+// that products of one phase can share the warps out (the FFMA path always uses every thread)
 template <bool TA, bool TB, bool kTC>
 __device__ __forceinline__ void bmm(float* C, int ldc, const float* A, int lda, const float* B, int ldb, int M, int N, int K,
-                    float alpha, bool accumulate) {
+                    float alpha, bool accumulate, int w0 = 0, int wn = kBwdThreads / 32) {
     if (kTC && M % 16 == 0 && N % 8 == 0 && K % 16 == 0) {
         if (K == 64)
-            bmm_mma<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+            bmm_mma<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate, w0, wn);
         else if (K == 16)
-            bmm_mma<TA, TB, 16>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+            bmm_mma<TA, TB, 16>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate, w0, wn);
         else
-            bmm_mma<TA, TB, 0>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
+            bmm_mma<TA, TB, 0>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate, w0, wn);
     } else if (K == 64)
         bmm_k<TA, TB, 64>(C, ldc, A, lda, B, ldb, M, N, K, alpha, accumulate);
     else if (K == 16)
@@ -416,16 +419,16 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             const int n = NC > 0 ? NC : n_rt;
             // ---- recompute the mini-batch's forward
             chunk_inner_grad<kTC>(m, n, d, eps);
-            bmm<false, true, kTC>(m.P, LDN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false);
+            // P = Q X^T (warps 8-15) and Q W, the first part of Zb = Q W + b - A G (warps 0-7, into tmp)
+            bmm<false, true, kTC>(m.P, LDN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false, 8, 8);
+            bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false, 0, 8);
             __syncthreads();
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
                 m.A[t * LDN + s_] = s_ <= t ? m.e[s_] * (m.P[t * LDN + s_] + 1.f) : 0.f;
             }
             __syncthreads();
-            // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb)
-            bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false);
-            __syncthreads();
+            // the rest of Zb (into tmp), z^ = LN0(Zb)
             bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true);
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
@@ -451,10 +454,12 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             ln_back_rows(m.dZb, m.zh, m.s2, n, d);
             __syncthreads();
             // ---- Zb = Q W + b - A G
-            bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true);      // dQ += dZb W^T
-            bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);    // dW_prev = Q^T dZb
-            bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
-            bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false);  // dG = -A^T dZb
+            bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dQ += dZb W^T
+            bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);       // dW_prev = Q^T dZb
+            bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false, 0, 2);  // dA = -(dZb G^T)
+            bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false, 2, 8);  // dG = -A^T dZb
+            // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp; -X dW here)
+            bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false, 8, 8);
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.dZb[t * LD + j];
@@ -465,8 +470,6 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 const int t = i / n, s_ = i % n;
                 if (s_ > t) m.dA[t * LDN + s_] = 0.f;
             }
-            // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp)
-            bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false);
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
@@ -486,23 +489,23 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                     if (lane == 0) m.de[t] = a + c;
                 }
             }
-            __syncthreads();  // tmp is read above and overwritten below
+            __syncthreads();  // tmp and dA are read above and overwritten below
             // dX = -(e G) dW^T  (tmp <- e G)
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, o = t * LD + i % d;
                 m.tmp[o] = m.e[t] * m.G[o];
             }
+            // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
+            for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
-            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false);
+            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false, 0, 8);
+            bmm<false, false, kTC>(m.dQc, LD, m.dA, LDN, m.X, LD, n, d, n, 1.f, true, 8, 8);   // dQ += dP X
             // dW_prev += dW (the state passes through)
             for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
                 const int o = (i / d) * LD + i % d;
                 m.dWp[o] += m.dW[o];
             }
-            // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
-            for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
-            bmm<false, false, kTC>(m.dQc, LD, m.dA, LDN, m.X, LD, n, d, n, 1.f, true);   // dQ += dP X
             bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
             // ---- G = s (Gx - m1 - x^ m2), Gx = 2 gamma R, R = X + gamma x^ + beta - V
             {
@@ -563,8 +566,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             }
             __syncthreads();
             // ---- Y = X W + b
-            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true);     // dX += dY W^T
-            bmm<true, false, kTC>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true);     // dW_prev += X^T dY
+            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dX += dY W^T
+            bmm<true, false, kTC>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true, 8, 8);  // dW_prev += X^T dY
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
