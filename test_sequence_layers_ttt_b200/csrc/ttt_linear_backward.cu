@@ -47,9 +47,6 @@ constexpr int kMaxD = 64, kMaxN = 16;
 constexpr int LD = kMaxD + 1;  // padded row length of every [rows][d] array
 constexpr int LDN = kMaxN + 1;  // padded row length of the [n][n] token-pair arrays
 
-template <typename T>
-__device__ __forceinline__ float ldv(const T* p, size_t i) { return to_f32(p[i]); }
-
 // C (=|+=) alpha * op(A) op(B), op(A)(i,k) = TA ? A[k][i] : A[i][k], op(B)(k,j) = TB ? B[j][k] : B[k][j].
 // Each thread owns a TM x TN block of C in registers, so every element it loads from shared memory
 // feeds TN (or TM) multiply-adds; M % TM == 0 and N % TN == 0.
@@ -262,7 +259,10 @@ template <typename T, bool kTokens, bool kBackward>
 struct Prefetch {
     static constexpr int kTok = kMaxN * kMaxD / kBwdThreads;  // 2
     static constexpr int kSt = kMaxD * kMaxD / kBwdThreads;   // 8
-    float x[kTok], q[kTok], v[kTok], dz[kTok], e, w[kSt], bb;
+    // the token rows are held as loaded (bf16 or fp32) and converted in commit(): a conversion
+    // here would make every warp wait for its loads before going on
+    T x[kTok], q[kTok], v[kTok];
+    float dz[kTok], e, w[kSt], bb;
     int n = 0;
 
     __device__ void issue(const T* Q, const T* K, const T* V, const float* eta, const float* dZ, const float* st,
@@ -274,9 +274,9 @@ struct Prefetch {
             const int i = tid + k * kBwdThreads;
             if (i < n * d) {
                 const size_t gi = base * d + i;
-                x[k] = ldv(K, gi);
-                q[k] = ldv(Q, gi);
-                v[k] = ldv(V, gi);
+                x[k] = K[gi];
+                q[k] = Q[gi];
+                v[k] = V[gi];
                 if (kBackward) dz[k] = dZ[gi];
             }
         }
@@ -297,9 +297,9 @@ struct Prefetch {
             const int i = tid + k * kBwdThreads;
             if (i < n * d) {
                 const int o = (i / d) * LD + i % d;
-                m.X[o] = x[k];
-                m.Qm[o] = q[k];
-                m.Vm[o] = v[k];
+                m.X[o] = to_f32(x[k]);
+                m.Qm[o] = to_f32(q[k]);
+                m.Vm[o] = to_f32(v[k]);
                 if (kBackward) m.dZ[o] = dz[k];
             }
         }
@@ -456,8 +456,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- Zb = Q W + b - A G
             bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dQ += dZb W^T
             bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);       // dW_prev = Q^T dZb
-            bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false, 0, 2);  // dA = -(dZb G^T)
-            bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false, 2, 8);  // dG = -A^T dZb
+            bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false, 8, 8);  // dG = -A^T dZb
             // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp; -X dW here)
             bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false, 8, 8);
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
@@ -466,11 +465,12 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 m.dbp[j] = a + m.db[j];
             }
             __syncthreads();
+            bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
+            __syncthreads();
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
                 if (s_ > t) m.dA[t * LDN + s_] = 0.f;
             }
-            __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
                 m.tmp[o] -= m.db[j];
