@@ -181,12 +181,17 @@ struct BwdSmem {
     float gam[kMaxD], bet[kMaxD], dgam[kMaxD], dbet[kMaxD];
 };
 
-// x^ = (y - mean y) s, s = (var y + eps)^(-1/2), per row of y [n][d]; one warp per row
-__device__ __forceinline__ void ln_rows(const float* y, float* xh, float* s, int n, int d, float eps) {
+// x^ = (y - mean y) s, s = (var y + eps)^(-1/2), per row of y + bias [n][d] (y updated in place to
+// y + bias); one warp per row
+__device__ __forceinline__ void ln_rows_bias(float* y, const float* bias, float* xh, float* s, int n, int d,
+                                             float eps) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int t = warp; t < n; t += nw) {
         float a = 0.f;
-        for (int j = lane; j < d; j += 32) a += y[t * LD + j];
+        for (int j = lane; j < d; j += 32) {
+            y[t * LD + j] += bias[j];
+            a += y[t * LD + j];
+        }
         const float mu = warp_sum(a) / d;
         float v = 0.f;
         for (int j = lane; j < d; j += 32) {
@@ -213,41 +218,50 @@ __device__ __forceinline__ void ln_back_rows(float* dxh, const float* xh, const 
     }
 }
 
-// Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G)
+// Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G).
+// After the product every step is local to a token row, so one warp per row runs them all
+// with no block barrier in between.
 template <bool kTC>
 __device__ __forceinline__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
     bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
     __syncthreads();
-    for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
-    __syncthreads();
-    ln_rows(m.tmp, m.xh, m.s, n, d, eps);
-    __syncthreads();
-    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-        const int t = i / d, j = i % d, o = t * LD + j;
-        m.R[o] = m.X[o] + m.gam[j] * m.xh[o] + m.bet[j] - m.Vm[o];
-        m.Gx[o] = 2.f * m.gam[j] * m.R[o];
-    }
-    __syncthreads();
-    {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-        for (int t = warp; t < n; t += nw) {
-            float a = 0.f, c = 0.f;
-            for (int j = lane; j < d; j += 32) {
-                a += m.Gx[t * LD + j];
-                c = fmaf(m.Gx[t * LD + j], m.xh[t * LD + j], c);
-            }
-            a = warp_sum(a) / d;
-            c = warp_sum(c) / d;
-            if (lane == 0) {
-                m.m1[t] = a;
-                m.m2[t] = c;
-            }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int t = warp; t < n; t += nw) {
+        float* y = m.tmp + t * LD;
+        float a = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            y[j] += m.b[j];
+            a += y[j];
         }
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-        const int t = i / d, o = t * LD + i % d;
-        m.G[o] = m.s[t] * (m.Gx[o] - m.m1[t] - m.xh[o] * m.m2[t]);
+        const float mu = warp_sum(a) / d;
+        float v = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            const float c = y[j] - mu;
+            v = fmaf(c, c, v);
+        }
+        const float rs = rsqrtf(warp_sum(v) / d + eps);
+        float s1 = 0.f, s2 = 0.f;
+        for (int j = lane; j < d; j += 32) {
+            const int o = t * LD + j;
+            const float xh = (y[j] - mu) * rs;
+            const float r = m.X[o] + m.gam[j] * xh + m.bet[j] - m.Vm[o];
+            const float gx = 2.f * m.gam[j] * r;
+            m.xh[o] = xh;
+            m.R[o] = r;
+            m.Gx[o] = gx;
+            s1 += gx;
+            s2 = fmaf(gx, xh, s2);
+        }
+        const float m1 = warp_sum(s1) / d, m2 = warp_sum(s2) / d;
+        for (int j = lane; j < d; j += 32) {
+            const int o = t * LD + j;
+            m.G[o] = rs * (m.Gx[o] - m1 - m.xh[o] * m2);
+        }
+        if (lane == 0) {
+            m.s[t] = rs;
+            m.m1[t] = m1;
+            m.m2[t] = m2;
+        }
     }
     __syncthreads();
 }
@@ -431,9 +445,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // the rest of Zb (into tmp), z^ = LN0(Zb)
             bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true);
             __syncthreads();
-            for (int i = threadIdx.x; i < n * d; i += blockDim.x) m.tmp[(i / d) * LD + i % d] += m.b[i % d];
-            __syncthreads();
-            ln_rows(m.tmp, m.zh, m.s2, n, d, eps);
+            ln_rows_bias(m.tmp, m.b, m.zh, m.s2, n, d, eps);
             __syncthreads();
             // ---- z = q + gamma z^ + beta
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
