@@ -204,20 +204,6 @@ __device__ __forceinline__ void ln_rows_bias(float* y, const float* bias, float*
     }
 }
 
-// dy = s (dx^ - mean dx^ - x^ mean(dx^ x^)) per row, in place on dxh
-__device__ __forceinline__ void ln_back_rows(float* dxh, const float* xh, const float* s, int n, int d) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int t = warp; t < n; t += nw) {
-        float a = 0.f, c = 0.f;
-        for (int j = lane; j < d; j += 32) {
-            a += dxh[t * LD + j];
-            c = fmaf(dxh[t * LD + j], xh[t * LD + j], c);
-        }
-        const float ma = warp_sum(a) / d, mc = warp_sum(c) / d;
-        for (int j = lane; j < d; j += 32) dxh[t * LD + j] = s[t] * (dxh[t * LD + j] - ma - xh[t * LD + j] * mc);
-    }
-}
-
 // Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G).
 // After the product every step is local to a token row, so one warp per row runs them all
 // with no block barrier in between.
@@ -457,13 +443,26 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 m.dgam[j] += a;
                 m.dbet[j] += c;
             }
-            for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-                const int o = (i / d) * LD + i % d;
-                m.dQc[o] = m.dZ[o];
-                m.dZb[o] = m.dZ[o] * m.gam[i % d];
+            // dQ = dZ (the residual); dZb = LNback(gamma dZ), one warp per row
+            {
+                const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+                for (int t = warp; t < n; t += nw) {
+                    float a = 0.f, c = 0.f;
+                    for (int j = lane; j < d; j += 32) {
+                        const int o = t * LD + j;
+                        const float g_ = m.dZ[o] * m.gam[j];
+                        m.dQc[o] = m.dZ[o];
+                        m.dZb[o] = g_;
+                        a += g_;
+                        c = fmaf(g_, m.zh[o], c);
+                    }
+                    const float ma = warp_sum(a) / d, mc = warp_sum(c) / d;
+                    for (int j = lane; j < d; j += 32) {
+                        const int o = t * LD + j;
+                        m.dZb[o] = m.s2[t] * (m.dZb[o] - ma - m.zh[o] * mc);
+                    }
+                }
             }
-            __syncthreads();
-            ln_back_rows(m.dZb, m.zh, m.s2, n, d);
             __syncthreads();
             // ---- Zb = Q W + b - A G
             bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dQ += dZb W^T
@@ -541,16 +540,32 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 }
             }
             __syncthreads();
-            // dGx (into dZb), dxh (into tmp), dR (into dG)
-            for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-                const int t = i / d, j = i % d, o = t * LD + j;
-                const float s_ = m.s[t];
-                const float dgx = s_ * (m.dG[o] - m.m1[t]) - s_ * m.mdg[t] * m.xh[o];
-                const float dxh = -s_ * m.m2[t] * m.dG[o] - s_ * m.mdg[t] * m.Gx[o];
-                const float dr = 2.f * m.gam[j] * dgx;
-                m.dZb[o] = dgx;
-                m.tmp[o] = dxh + m.gam[j] * dr;
-                m.dG[o] = dr;
+            // dGx (into dZb), dR (into dG), and dY = LNback(dxh) - ds s^2 x^ / d (into tmp): x^ = LN0(Y),
+            // and s appears explicitly in G; one warp per row
+            {
+                const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+                for (int t = warp; t < n; t += nw) {
+                    const float s_ = m.s[t];
+                    float a = 0.f, c = 0.f;
+                    for (int j = lane; j < d; j += 32) {
+                        const int o = t * LD + j;
+                        const float dgx = s_ * (m.dG[o] - m.m1[t]) - s_ * m.mdg[t] * m.xh[o];
+                        const float dxh = -s_ * m.m2[t] * m.dG[o] - s_ * m.mdg[t] * m.Gx[o];
+                        const float dr = 2.f * m.gam[j] * dgx;
+                        const float dx = dxh + m.gam[j] * dr;
+                        m.dZb[o] = dgx;
+                        m.tmp[o] = dx;
+                        m.dG[o] = dr;
+                        a += dx;
+                        c = fmaf(dx, m.xh[o], c);
+                    }
+                    const float ma = warp_sum(a) / d, mc = warp_sum(c) / d;
+                    for (int j = lane; j < d; j += 32) {
+                        const int o = t * LD + j;
+                        m.tmp[o] = s_ * (m.tmp[o] - ma - m.xh[o] * mc);
+                        m.tmp[o] -= m.ds[t] * s_ * s_ * m.xh[o] * inv_d;
+                    }
+                }
             }
             __syncthreads();
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
@@ -567,14 +582,6 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 const int t = i / d, j = i % d, o = t * LD + j;
                 m.dXc[o] += m.dG[o];
                 dV[(base + t) * d + j] = -m.dG[o];
-            }
-            __syncthreads();
-            // x^ = LN0(Y), and s appears explicitly in G: dY = LNback(dxh) - ds s^2 x^ / d  (into tmp)
-            ln_back_rows(m.tmp, m.xh, m.s, n, d);
-            __syncthreads();
-            for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
-                const int t = i / d, o = t * LD + i % d;
-                m.tmp[o] -= m.ds[t] * m.s[t] * m.s[t] * m.xh[o] * inv_d;
             }
             __syncthreads();
             // ---- Y = X W + b
