@@ -105,7 +105,7 @@ def ttt_linear_backward(Q, K, V, eta, W0, b0, gamma, beta, dZ, mini_batch: int,
 
     ``dtype=torch.float32`` evaluates the same steps in single precision: not a
     reference, but the rounding floor of any fp32 implementation of the scan's
-    backward, against which a long sequence's fp32 errors are judged."""
+    backward, which sets the bar for a long sequence's fp32 errors."""
     plain = mode == MODE_PLAIN
     c = lambda x, rg=False: _t(x, rg, dtype)
     Qt, Kt, Vt, et, W0t = (c(x, True) for x in (Q, K, V, eta, W0))

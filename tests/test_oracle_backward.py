@@ -82,8 +82,8 @@ def test_gradients_equal_finite_differences_of_the_c_oracle(mode, mb):
 
 
 def test_float32_evaluation_is_the_same_algorithm():
-    """The backward oracle's single-precision evaluation (the fp32 floor used to
-    judge long sequences) runs the same steps: on a short, well-conditioned case
+    """The backward oracle's single-precision evaluation (the fp32 floor that sets
+    the bar for long sequences) runs the same steps: on a short, well-conditioned case
     it agrees with the float64 result to single-precision rounding, and its
     outputs are float32."""
     import torch
