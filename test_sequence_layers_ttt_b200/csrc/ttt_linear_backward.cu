@@ -406,6 +406,12 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
         pf.issue(Q, K, V, eta, dZ, states + ((size_t)bh * nmb + jb) * sz, (size_t)bh * T_ + t0, min(mb, T_ - t0),
                  d);
     };
+    // the carried gradient of the state (dW, db) and the one being formed for the state before the
+    // current mini-batch (dW_prev, db_prev)
+    float* cW = m.dW;
+    float* cWp = m.dWp;
+    float* cb = m.db;
+    float* cbp = m.dbp;
     if (nmb > 0) issue(nmb - 1);
     for (int jb = nmb - 1; jb >= 0; jb--) {
         const int t0 = jb * mb, n_rt = min(mb, T_ - t0);
@@ -466,14 +472,14 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             __syncthreads();
             // ---- Zb = Q W + b - A G
             bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dQ += dZb W^T
-            bmm<true, false, kTC>(m.dWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);       // dW_prev = Q^T dZb
+            bmm<true, false, kTC>(cWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);       // dW_prev = Q^T dZb
             bmm<true, false, kTC>(m.dG, LD, m.A, LDN, m.dZb, LD, n, d, n, -1.f, false, 8, 8);  // dG = -A^T dZb
             // ---- W' = W - X^T diag(e) G, b' = b - G^T e:  dEG = -(X dW) - db (into tmp; -X dW here)
-            bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.dW, LD, n, d, d, -1.f, false, 8, 8);
+            bmm<false, false, kTC>(m.tmp, LD, m.X, LD, cW, LD, n, d, d, -1.f, false, 8, 8);
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.dZb[t * LD + j];
-                m.dbp[j] = a + m.db[j];
+                cbp[j] = a + cb[j];
             }
             __syncthreads();
             bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
@@ -484,7 +490,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             }
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
-                m.tmp[o] -= m.db[j];
+                m.tmp[o] -= cb[j];
                 m.dG[o] = fmaf(m.e[t], m.tmp[o], m.dG[o]);
             }
             __syncthreads();
@@ -509,12 +515,12 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
-            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.dW, LD, n, d, d, -1.f, false, 0, 8);
+            bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, cW, LD, n, d, d, -1.f, false, 0, 8);
             bmm<false, false, kTC>(m.dQc, LD, m.dA, LDN, m.X, LD, n, d, n, 1.f, true, 8, 8);   // dQ += dP X
             // dW_prev += dW (the state passes through)
             for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
                 const int o = (i / d) * LD + i % d;
-                m.dWp[o] += m.dW[o];
+                cWp[o] += cW[o];
             }
             __syncthreads();
             bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
@@ -586,11 +592,11 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             __syncthreads();
             // ---- Y = X W + b
             bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dX += dY W^T
-            bmm<true, false, kTC>(m.dWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true, 8, 8);  // dW_prev += X^T dY
+            bmm<true, false, kTC>(cWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true, 8, 8);  // dW_prev += X^T dY
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f;
                 for (int t = 0; t < n; t++) a += m.tmp[t * LD + j];
-                m.dbp[j] += a;
+                cbp[j] += a;
             }
             __syncthreads();
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
@@ -599,21 +605,24 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 dK[(base + t) * d + j] = m.dXc[o];
             }
             for (int t = threadIdx.x; t < n; t += blockDim.x) deta[base + t] = m.de[t];
-            for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
-                const int o = (i / d) * LD + i % d;
-                m.dW[o] = m.dWp[o];
-            }
-            for (int j = threadIdx.x; j < d; j += blockDim.x) m.db[j] = m.dbp[j];
-            __syncthreads();
+            // the gradient of the state before this mini-batch becomes the carried one: the two
+            // buffers swap roles (the next mini-batch overwrites cWp, cbp before reading them)
+            float* const sw = cW;
+            cW = cWp;
+            cWp = sw;
+            float* const sb = cb;
+            cb = cbp;
+            cbp = sb;
         };
         if (n_rt == kMaxN)
             chunk(std::integral_constant<int, kMaxN>{});
         else
             chunk(std::integral_constant<int, 0>{});
     }
-    for (int i = threadIdx.x; i < d * d; i += blockDim.x) dW0[(size_t)bh * d * d + i] = m.dW[(i / d) * LD + i % d];
+    __syncthreads();
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) dW0[(size_t)bh * d * d + i] = cW[(i / d) * LD + i % d];
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        db0[(size_t)bh * d + j] = m.db[j];
+        db0[(size_t)bh * d + j] = cb[j];
         gb_partial[((size_t)bh * 2 + 0) * d + j] = m.dgam[j];
         gb_partial[((size_t)bh * 2 + 1) * d + j] = m.dbet[j];
     }
