@@ -204,12 +204,13 @@ __device__ __forceinline__ void ln_rows_bias(float* y, const float* bias, float*
     }
 }
 
-// Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G).
-// After the product every step is local to a token row, so one warp per row runs them all
-// with no block barrier in between.
-template <bool kTC>
+// Y = X W + b into tmp; x^, s; R, Gx, m1, m2, G (the forward of one mini-batch up to G); with kWithA
+// also P = Q X^T and A = tril(e_s (P + 1)).  After the products every step is local to a token row,
+// so one warp per row runs them all with no block barrier in between.
+template <bool kTC, bool kWithA>
 __device__ __forceinline__ void chunk_inner_grad(BwdSmem& m, int n, int d, float eps) {
-    bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);
+    bmm<false, false, kTC>(m.tmp, LD, m.X, LD, m.W, LD, n, d, d, 1.f, false);  // 8 tiles: warps 0-7
+    if (kWithA) bmm<false, true, kTC>(m.P, LDN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false, 8, 8);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int t = warp; t < n; t += nw) {
@@ -248,6 +249,7 @@ __device__ __forceinline__ void chunk_inner_grad(BwdSmem& m, int n, int d, float
             m.m1[t] = m1;
             m.m2[t] = m2;
         }
+        if (kWithA && lane < n) m.A[t * LDN + lane] = lane <= t ? m.e[lane] * (m.P[t * LDN + lane] + 1.f) : 0.f;
     }
     __syncthreads();
 }
@@ -352,7 +354,7 @@ ttt_linear_states_kernel(int T_, int d_arg, int mb, float eps, const T* Q, const
         auto chunk = [&](auto nc) {
             constexpr int NC = decltype(nc)::value;
             const int n = NC > 0 ? NC : n_rt;
-            chunk_inner_grad<kTC>(m, n, d, eps);
+            chunk_inner_grad<kTC, false>(m, n, d, eps);
             // W -= X^T diag(e) G, b -= G^T e
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, o = t * LD + i % d;
@@ -424,18 +426,12 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             constexpr int NC = decltype(nc)::value;
             const int n = NC > 0 ? NC : n_rt;
             // ---- recompute the mini-batch's forward
-            chunk_inner_grad<kTC>(m, n, d, eps);
-            // P = Q X^T (warps 8-15) and Q W, the first part of Zb = Q W + b - A G (warps 0-7, into tmp)
-            bmm<false, true, kTC>(m.P, LDN, m.Qm, LD, m.X, LD, n, n, d, 1.f, false, 8, 8);
+            chunk_inner_grad<kTC, true>(m, n, d, eps);  // also P = Q X^T and A
+            // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb).  The two products give each 16 x 8 tile of C to
+            // the same warp (off the tensor cores, each element to the same thread), so the second
+            // follows the first without a barrier.
             bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false, 0, 8);
-            __syncthreads();
-            for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
-                const int t = i / n, s_ = i % n;
-                m.A[t * LDN + s_] = s_ <= t ? m.e[s_] * (m.P[t * LDN + s_] + 1.f) : 0.f;
-            }
-            __syncthreads();
-            // the rest of Zb (into tmp), z^ = LN0(Zb)
-            bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true);
+            bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true, 0, 8);
             __syncthreads();
             ln_rows_bias(m.tmp, m.b, m.zh, m.s2, n, d, eps);
             __syncthreads();
@@ -515,15 +511,15 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
+            // dX = -(e G) dW^T + dP^T Q (the same tiles on the same warps, so no barrier between them)
             bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, cW, LD, n, d, d, -1.f, false, 0, 8);
+            bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true, 0, 8);
             bmm<false, false, kTC>(m.dQc, LD, m.dA, LDN, m.X, LD, n, d, n, 1.f, true, 8, 8);   // dQ += dP X
             // dW_prev += dW (the state passes through)
             for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
                 const int o = (i / d) * LD + i % d;
                 cWp[o] += cW[o];
             }
-            __syncthreads();
-            bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true);   // dX += dP^T Q
             // ---- G = s (Gx - m1 - x^ m2), Gx = 2 gamma R, R = X + gamma x^ + beta - V
             {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
