@@ -121,6 +121,43 @@ def test_linear_backward_long_sequence(ttt):
         assert err <= bar, f"{name}: max err {err:.2e} of RMS > {bar:.2e} (fp32 floor {floor:.2e})"
 
 
+@pytest.fixture(scope="module")
+def full_size_run(ttt):
+    """The whole 1.3B-layer workload at 32k tokens (B = 2, H = 32: the bench's launch), run once."""
+    w = WORKLOADS["linear_1p3b_32k"]
+    inp = make_inputs(w, 0)
+    dZ, dW, db = upstream(w, 0)
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    got = ttt.ttt_linear_backward(*(inp[k].cuda() for k in keys), dZ.cuda(), dW.cuda(), db.cuda(), mini_batch=16,
+                                  ln_eps=w.ln_eps)
+    torch.cuda.synchronize()
+    return w, inp, (dZ, dW, db), [g.cpu() for g in got[:6]]
+
+
+@pytest.mark.parametrize("scan", [(0, 5), (1, 27)])
+def test_linear_backward_full_size_sampled_scans(full_size_run, scan):
+    """The per-scan gradients (dQ, dK, dV, deta, dW0, db0) of one sampled (batch, head) scan of
+    the full-size run, checked against the oracle run on that scan alone (the scans are
+    independent; dgamma, dbeta, sums over the batch, are left to the smaller cases).  Bar:
+    four times the fp32 floor of that scan, never below 1e-3."""
+    w, inp, (dZ, dW, db), got = full_size_run
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    b, h = scan
+    one = {k: inp[k][b:b + 1, h:h + 1] for k in ("Q", "K", "V", "eta", "W0", "b0")}
+    one.update({k: inp[k][h:h + 1] for k in ("gamma", "beta")})
+    sl = lambda t: t[b:b + 1, h:h + 1]
+    args = [one[k] for k in keys]
+    ref = ob.ttt_linear_backward(*args, sl(dZ), 16, ln_eps=w.ln_eps, dW_T=sl(dW), db_T=sl(db))
+    f32 = ob.ttt_linear_backward(*args, sl(dZ), 16, ln_eps=w.ln_eps, dW_T=sl(dW), db_T=sl(db), dtype=torch.float32)
+    for name, a, r, f in zip(NAMES[:6], got, ref, f32):
+        a = sl(a).numpy().astype(np.float64)
+        assert np.isfinite(a).all(), f"{name}: non-finite"
+        floor = float(np.abs(np.asarray(f, dtype=np.float64) - r).max()) / rms(r)
+        err = float(np.abs(a - r).max()) / rms(r)
+        bar = max(BAR, FLOOR_FACTOR * floor)
+        assert err <= bar, f"{name}: max err {err:.2e} of RMS > {bar:.2e} (fp32 floor {floor:.2e})"
+
+
 def test_linear_backward_empty_sequence(ttt):
     """T = 0: dW0 = dW_T, db0 = db_T, dgamma = dbeta = 0."""
     w = WORKLOADS["linear_125m_2k"].with_shape(B=1, H=2, T=0)
