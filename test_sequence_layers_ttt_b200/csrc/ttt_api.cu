@@ -456,12 +456,15 @@ int ttt_abi_version(void) { return 103; }
 
 #ifdef TTT_TIMELINE
 // Timeline builds only (not part of the ABI): copy the clock64 stamps of CTA 0
-// of the last launch of kernel `which` (0: ttt_linear_lag_kernel) into
+// of the last launch of kernel `which` (0: ttt_linear_lag_kernel, 1: the backward's
+// ttt_linear_backward_kernel) into
 // out[kTlRoles][kTlChunks][kTlEvents].
 int ttt_debug_timeline(int which, long long* out) {
     if (!out) return TTT_ERR_NULL;
     if (cudaDeviceSynchronize() != cudaSuccess) return TTT_ERR_CUDA;
-    const cudaError_t e = which == 0 ? ttt::read_lag_timeline(out) : cudaErrorInvalidValue;
+    const cudaError_t e = which == 0   ? ttt::read_lag_timeline(out)
+                          : which == 1 ? ttt::read_bwd_timeline(out)
+                                       : cudaErrorInvalidValue;
     return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 #endif

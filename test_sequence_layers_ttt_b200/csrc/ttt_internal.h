@@ -101,6 +101,7 @@ cudaError_t read_and_clear_mlp_error(unsigned int* out);
 cudaError_t read_and_clear_device_error(unsigned int* out);
 #ifdef TTT_TIMELINE
 cudaError_t read_lag_timeline(long long* out);     // kTlRoles x kTlChunks x kTlEvents stamps
+cudaError_t read_bwd_timeline(long long* out);     // the same layout, the backward's reverse sweep
 #endif
 
 // Fault-injection hook: the chunk index named by TTT_DEBUG_DROP_CHUNK (read once

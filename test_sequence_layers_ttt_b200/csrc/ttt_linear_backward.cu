@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "timeline.cuh"
 #include "ttt_internal.h"
 
 namespace ttt {
@@ -38,6 +39,9 @@ namespace ttt {
 // Workspace of ttt_linear_backward_static: a fixed array that every device
 // loading the library holds until the process exits, for callers that cannot
 // allocate device memory.  Shared by every call on a device.
+// clock64 stamps of the reverse sweep (TTT_TIMELINE builds only): 16 points per mini-batch
+TTT_TIMELINE_BUFFER(g_bwd_timeline);
+
 static __device__ __align__(256) unsigned char g_backward_static_workspace[kBackwardStaticWorkspaceBytes];
 
 namespace {
@@ -385,6 +389,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                            float* dW0, float* db0, float* gb_partial) {
     extern __shared__ float smem_f[];
     BwdSmem& m = *reinterpret_cast<BwdSmem*>(smem_f);
+    TTT_TIMELINE_SMEM();
     constexpr int d = DT;
     constexpr bool kTC = DT == 64;  // products on the tensor cores
     (void)d_arg;
@@ -414,17 +419,26 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
     float* cWp = m.dWp;
     float* cb = m.db;
     float* cbp = m.dbp;
+    // point k of mini-batch jb's step (CTA 0, TTT_TIMELINE builds; nothing otherwise)
+    auto stamp = [&](int jb_, int k) {
+        TTT_STAMP(g_bwd_timeline, threadIdx.x == 0, k >> 3, nmb - 1 - jb_, k & 7);
+        (void)jb_;
+        (void)k;
+    };
     if (nmb > 0) issue(nmb - 1);
     for (int jb = nmb - 1; jb >= 0; jb--) {
         const int t0 = jb * mb, n_rt = min(mb, T_ - t0);
         const size_t base = (size_t)bh * T_ + t0;
         pf.commit(m, d);
+        stamp(jb, 14);
         if (jb > 0) issue(jb - 1);
+        stamp(jb, 15);
         __syncthreads();
         // full mini-batches take a copy of the body with n fixed at compile time
         auto chunk = [&](auto nc) {
             constexpr int NC = decltype(nc)::value;
             const int n = NC > 0 ? NC : n_rt;
+            stamp(jb, 0);
             // ---- recompute the mini-batch's forward
             chunk_inner_grad<kTC, true>(m, n, d, eps);  // also P = Q X^T and A
             // Zb = Q W + b - A G (into tmp), z^ = LN0(Zb).  The two products give each 16 x 8 tile of C to
@@ -433,8 +447,10 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             bmm<false, false, kTC>(m.tmp, LD, m.Qm, LD, m.W, LD, n, d, d, 1.f, false, 0, 8);
             bmm<false, false, kTC>(m.tmp, LD, m.A, LDN, m.G, LD, n, d, n, -1.f, true, 0, 8);
             __syncthreads();
+            stamp(jb, 1);
             ln_rows_bias(m.tmp, m.b, m.zh, m.s2, n, d, eps);
             __syncthreads();
+            stamp(jb, 2);
             // ---- z = q + gamma z^ + beta
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f, c = 0.f;
@@ -466,6 +482,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 }
             }
             __syncthreads();
+            stamp(jb, 3);
             // ---- Zb = Q W + b - A G
             bmm<false, true, kTC>(m.dQc, LD, m.dZb, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dQ += dZb W^T
             bmm<true, false, kTC>(cWp, LD, m.Qm, LD, m.dZb, LD, d, d, n, 1.f, false);       // dW_prev = Q^T dZb
@@ -478,8 +495,10 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 cbp[j] = a + cb[j];
             }
             __syncthreads();
+            stamp(jb, 4);
             bmm<false, true, kTC>(m.dA, LDN, m.dZb, LD, m.G, LD, n, n, d, -1.f, false);  // dA = -(dZb G^T)
             __syncthreads();
+            stamp(jb, 5);
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) {
                 const int t = i / n, s_ = i % n;
                 if (s_ > t) m.dA[t * LDN + s_] = 0.f;
@@ -490,6 +509,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 m.dG[o] = fmaf(m.e[t], m.tmp[o], m.dG[o]);
             }
             __syncthreads();
+            stamp(jb, 6);
             {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
                 for (int t = warp; t < n; t += nw) {  // de = sum_j dEG G + sum_t dA (P + 1)
@@ -503,6 +523,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 }
             }
             __syncthreads();  // tmp and dA are read above and overwritten below
+            stamp(jb, 7);
             // dX = -(e G) dW^T  (tmp <- e G)
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, o = t * LD + i % d;
@@ -511,6 +532,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
+            stamp(jb, 8);
             // dX = -(e G) dW^T + dP^T Q (the same tiles on the same warps, so no barrier between them)
             bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, cW, LD, n, d, d, -1.f, false, 0, 8);
             bmm<true, false, kTC>(m.dXc, LD, m.dA, LDN, m.Qm, LD, n, d, n, 1.f, true, 0, 8);
@@ -542,6 +564,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 }
             }
             __syncthreads();
+            stamp(jb, 9);
             // dGx (into dZb), dR (into dG), and dY = LNback(dxh) - ds s^2 x^ / d (into tmp): x^ = LN0(Y),
             // and s appears explicitly in G; one warp per row
             {
@@ -570,6 +593,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 }
             }
             __syncthreads();
+            stamp(jb, 10);
             for (int j = threadIdx.x; j < d; j += blockDim.x) {
                 float a = 0.f, c = 0.f;
                 for (int t = 0; t < n; t++) {
@@ -586,6 +610,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 dV[(base + t) * d + j] = -m.dG[o];
             }
             __syncthreads();
+            stamp(jb, 11);
             // ---- Y = X W + b
             bmm<false, true, kTC>(m.dXc, LD, m.tmp, LD, m.W, LD, n, d, d, 1.f, true, 0, 8);  // dX += dY W^T
             bmm<true, false, kTC>(cWp, LD, m.X, LD, m.tmp, LD, d, d, n, 1.f, true, 8, 8);  // dW_prev += X^T dY
@@ -595,6 +620,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 cbp[j] += a;
             }
             __syncthreads();
+            stamp(jb, 12);
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
                 dQ[(base + t) * d + j] = m.dQc[o];
@@ -609,6 +635,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             float* const sb = cb;
             cb = cbp;
             cbp = sb;
+            stamp(jb, 13);
         };
         if (n_rt == kMaxN)
             chunk(std::integral_constant<int, kMaxN>{});
@@ -616,6 +643,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             chunk(std::integral_constant<int, 0>{});
     }
     __syncthreads();
+    for (int r = 0; r < 2; r++) TTT_TIMELINE_FLUSH(g_bwd_timeline, threadIdx.x == 0, r);
     for (int i = threadIdx.x; i < d * d; i += blockDim.x) dW0[(size_t)bh * d * d + i] = cW[(i / d) * LD + i % d];
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         db0[(size_t)bh * d + j] = cb[j];
@@ -734,3 +762,11 @@ float* backward_static_workspace() {
 }
 
 }  // namespace ttt
+
+#ifdef TTT_TIMELINE
+namespace ttt {
+cudaError_t read_bwd_timeline(long long* out) {
+    return cudaMemcpyFromSymbol(out, g_bwd_timeline, sizeof(g_bwd_timeline));
+}
+}  // namespace ttt
+#endif

@@ -9,6 +9,7 @@ time between the role's stamped points, and the median time from the chain's
 hand-off of chunk c to each consumer's pick-up.
 
     python -m test_sequence_layers_ttt_b200.timeline [tensorcore]
+    python -m test_sequence_layers_ttt_b200.timeline backward   # the layer backward's reverse sweep
 
 Needs a GPU.  The stamps perturb the kernel a little (one clock read and one
 store per point, CTA 0 only).
@@ -35,6 +36,54 @@ ROLES = {
     }),
 }
 N_ROLES, N_CHUNKS, N_EVENTS, FIRST = 8, 32, 8, 1024
+
+# The layer backward's reverse sweep (one CTA per (batch, head), all threads in step): stamp k of a
+# mini-batch after the phase named here, in the order they run.
+BACKWARD_POINTS = [
+    (14, "commit of the prefetched inputs"), (15, "next mini-batch's loads issued"), (0, "barrier"),
+    (1, "forward recomputed (2 products, 1 row pass) + Zb products"), (2, "output LayerNorm rows"),
+    (3, "dgamma/dbeta; dQ = dZ; dZb (row pass)"), (4, "dZb products (dQ, dW_prev, dG, -X dW) + db_prev"),
+    (5, "dA product"), (6, "dA mask; dEG; dG += e dEG"), (7, "de rows"), (8, "tmp = e G; dP = dA e"),
+    (9, "dX, dQ products; dW_prev += dW; dG row sums"), (10, "row pass: dGx, dR, dY"),
+    (11, "dgamma/dbeta; dX += dR; dV"), (12, "dY products + db_prev"), (13, "stores of dQ, dK, deta; swap"),
+]
+
+
+def backward() -> None:
+    """The reverse sweep's per-mini-batch phases (1.3B shape, CTA 0, mini-batches 1024..1055 of the
+    sweep)."""
+    from test_sequence_layers_ttt_b200 import build as lib_build
+    os.environ["TTT_B200_LIBRARY"] = lib_build.build(timeline=True)
+    import torch
+    from test_sequence_layers_ttt_b200 import _binding as ttt
+    from test_sequence_layers_ttt_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS["linear_1p3b_32k"]
+    g = {k: v.cuda() for k, v in make_inputs(w, 0).items()}
+    gen = torch.Generator().manual_seed(0)
+    dZ = torch.randn((w.B, w.H, w.T, w.d), generator=gen).cuda()
+    keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
+    for _ in range(2):
+        ttt.ttt_linear_backward(*(g[k] for k in keys), dZ, None, None, mini_batch=16, ln_eps=w.ln_eps)
+    torch.cuda.synchronize()
+    buf = np.zeros((N_ROLES, N_CHUNKS, N_EVENTS), dtype=np.int64)
+    fn = ttt.lib.ttt_debug_timeline
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    st = fn(1, buf.ctypes.data)
+    if st != 0:
+        raise RuntimeError(f"ttt_debug_timeline failed with status {st}")
+    at = lambda k: buf[k >> 3, :, k & 7].astype(np.float64)
+    period = np.median(np.diff(at(0)))
+    print(f"backward reverse sweep: CTA 0, mini-batches {FIRST}..{FIRST + N_CHUNKS - 1} of the sweep, "
+          f"SM cycles (median)")
+    print(f"  period per mini-batch {period:.0f}")
+    # each point's interval starts at the point before it; the commit's at the end (13) of the
+    # previous mini-batch
+    order = [k for k, _ in BACKWARD_POINTS]
+    for i, (k, label) in enumerate(BACKWARD_POINTS):
+        start = at(13)[:-1] if i == 0 else at(order[i - 1])[1:]
+        print(f"  {np.median(at(k)[1:] - start):7.0f}  {label}")
 
 
 def main(family: str = "tensorcore") -> None:
@@ -87,4 +136,7 @@ def main(family: str = "tensorcore") -> None:
 
 
 if __name__ == "__main__":
-    main(sys.argv[1] if len(sys.argv) > 1 else "tensorcore")
+    if len(sys.argv) > 1 and sys.argv[1] == "backward":
+        backward()
+    else:
+        main(sys.argv[1] if len(sys.argv) > 1 else "tensorcore")
