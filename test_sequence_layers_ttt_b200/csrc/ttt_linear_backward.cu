@@ -8,7 +8,8 @@
 // computes the gradients of  sum(Z dZ) + sum(W_T dW_T) + sum(b_T db_T)  with
 // respect to Q, K, V, eta, W0, b0, gamma and beta.
 //
-// Two passes, one CTA per (batch, head), fp32 in shared memory:
+// Two passes, one CTA per (batch, head), the mini-batch's arrays in fp32 in shared memory (for d = 64
+// the block products run on the tensor cores: mma.sync with bf16 hi/lo operands, fp32 accumulation):
 //   1. the forward scan records the state each mini-batch starts from, W_j
 //      (d x d) and b_j, in the caller's workspace (d^2 + d floats per
 //      mini-batch and head): the tensor-core scan kernel's checkpoint variant
@@ -36,12 +37,12 @@
 
 namespace ttt {
 
-// Workspace of ttt_linear_backward_static: a fixed array that every device
-// loading the library holds until the process exits, for callers that cannot
-// allocate device memory.  Shared by every call on a device.
 // clock64 stamps of the reverse sweep (TTT_TIMELINE builds only): 16 points per mini-batch
 TTT_TIMELINE_BUFFER(g_bwd_timeline);
 
+// Workspace of ttt_linear_backward_static: a fixed array that every device
+// loading the library holds until the process exits, for callers that cannot
+// allocate device memory.  Shared by every call on a device.
 static __device__ __align__(256) unsigned char g_backward_static_workspace[kBackwardStaticWorkspaceBytes];
 
 namespace {
@@ -529,6 +530,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
                 const int t = i / d, o = t * LD + i % d;
                 m.tmp[o] = m.e[t] * m.G[o];
             }
+            for (int t = threadIdx.x; t < n; t += blockDim.x) deta[base + t] = m.de[t];  // final
             // ---- A = tril(e_s (P + 1)), P = Q X^T:  dP = dA e_s (into dA)
             for (int i = threadIdx.x; i < n * n; i += blockDim.x) m.dA[(i / n) * LDN + i % n] *= m.e[i % n];
             __syncthreads();
@@ -570,6 +572,7 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
                 for (int t = warp; t < n; t += nw) {
+                    for (int j = lane; j < d; j += 32) dQ[(base + t) * d + j] = m.dQc[t * LD + j];  // final
                     const float s_ = m.s[t];
                     float a = 0.f, c = 0.f;
                     for (int j = lane; j < d; j += 32) {
@@ -623,10 +626,8 @@ ttt_linear_backward_kernel(int T_, int d_arg, int mb, float eps, const T* Q, con
             stamp(jb, 12);
             for (int i = threadIdx.x; i < n * d; i += blockDim.x) {
                 const int t = i / d, j = i % d, o = t * LD + j;
-                dQ[(base + t) * d + j] = m.dQc[o];
                 dK[(base + t) * d + j] = m.dXc[o];
             }
-            for (int t = threadIdx.x; t < n; t += blockDim.x) deta[base + t] = m.de[t];
             // the gradient of the state before this mini-batch becomes the carried one: the two
             // buffers swap roles (the next mini-batch overwrites cWp, cbp before reading them)
             float* const sw = cW;
