@@ -100,11 +100,11 @@ def test_linear_backward_125m_heads(ttt):
 FLOOR_FACTOR = 4.0
 
 
-def test_linear_backward_long_sequence(ttt):
-    """One head of the 1.3B-layer shape over 4096 tokens (256 mini-batches)."""
-    w = WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=1, T=4096)
-    inp = make_inputs(w, 2)
-    dZ, dW, db = upstream(w, 2)
+def check_against_float32_floor(ttt, w, seed):
+    """Past 16 mini-batches the bar is FLOOR_FACTOR times the error of the
+    oracle's own steps evaluated in float32, and never below BAR."""
+    inp = make_inputs(w, seed)
+    dZ, dW, db = upstream(w, seed)
     keys = ("Q", "K", "V", "eta", "W0", "b0", "gamma", "beta")
     got = ttt.ttt_linear_backward(*(inp[k].cuda() for k in keys), dZ.cuda(), dW.cuda(), db.cuda(), mini_batch=16,
                                   ln_eps=w.ln_eps)
@@ -119,6 +119,21 @@ def test_linear_backward_long_sequence(ttt):
         err = float(np.abs(a - r).max()) / rms(r)
         bar = max(BAR, FLOOR_FACTOR * floor)
         assert err <= bar, f"{name}: max err {err:.2e} of RMS > {bar:.2e} (fp32 floor {floor:.2e})"
+
+
+def test_linear_backward_long_sequence(ttt):
+    """One head of the 1.3B-layer shape over 4096 tokens (256 mini-batches)."""
+    check_against_float32_floor(ttt, WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=1, T=4096), 2)
+
+
+@pytest.mark.parametrize("T", [1008, 1000])
+def test_linear_backward_odd_and_ragged_mini_batch_counts(ttt, T):
+    """Three heads of the 1.3B-layer shape.  T = 1008 is 63 whole mini-batches,
+    an odd count and a multiple of none of the tensor-core checkpoint pass's
+    ring depths (4 and 8), so its rings end part-way through a cycle.  T = 1000
+    ends in a ragged mini-batch of 8 tokens: the checkpoints come from the fp32
+    pass, and the reverse sweep starts on a short block."""
+    check_against_float32_floor(ttt, WORKLOADS["linear_1p3b_32k"].with_shape(B=1, H=3, T=T), 3)
 
 
 @pytest.fixture(scope="module")
