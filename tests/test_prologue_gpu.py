@@ -42,14 +42,18 @@ def check(ttt, B, T, H, dm, seed, pos0=0, rotary=True, eta_base=1.0):
     torch.cuda.synchronize()
     ref = op.project(x.float(), tq.float(), tk.float(), tv.float(), tl.float(), bl, eta_base=eta_base,
                      rotary=rotary, pos0=pos0)
+    compare(out, ref)
+
+
+def compare(out, ref, where=""):
     for name, a, r in zip(("Q", "K", "V"), out[:3], ref[:3]):
         a = a.float().cpu().numpy().astype(np.float64)
         rms = float(np.sqrt(np.mean(r ** 2)))
         err = np.abs(a - r) - (2.0 ** -8) * np.abs(r) - 1e-5 * rms
-        assert err.max() <= 0, f"{name}: worst excess {err.max():.3e} (rms {rms:.3e})"
+        assert err.max() <= 0, f"{name}{where}: worst excess {err.max():.3e} (rms {rms:.3e})"
     e = out[3].cpu().numpy().astype(np.float64)
     rel = float(np.abs(e - ref[3]).max() / np.abs(ref[3]).max())
-    assert rel <= 1e-5, f"eta: {rel:.2e}"
+    assert rel <= 1e-5, f"eta{where}: {rel:.2e}"
 
 
 @pytest.mark.parametrize("B,T,H,dm,pos0", [
@@ -76,3 +80,21 @@ def test_prologue_refuses_unsupported_shapes(ttt):
     with pytest.raises(ttt.TTTError) as ei:
         ttt.ttt_prologue_forward(x.cuda(), tq.cuda(), tk.cuda(), tv.cuda(), tl.cuda(), bl.cuda())
     assert ei.value.status == 6
+
+
+def test_prologue_full_size_sampled_windows(ttt):
+    """The 1.3B layer at 32k tokens in one launch (B = 2, T = 32768, d_model
+    2048, H = 32: about 1.1 GB in and out).  Windows of 64 tokens in both
+    sequences are checked against the oracle run on each window alone at its
+    absolute position: the first window of the second sequence starts at GEMM
+    row 32768, where positions restart at 0."""
+    B, T, H, dm, W = 2, 32768, 32, 2048, 64
+    x, tq, tk, tv, tl, bl = make(B, T, H, dm, 5)
+    out = ttt.ttt_prologue_forward(x.cuda(), tq.cuda(), tk.cuda(), tv.cuda(), tl.cuda(), bl.cuda())
+    torch.cuda.synchronize()
+    weights = (tq.float(), tk.float(), tv.float(), tl.float(), bl)
+    for b in range(B):
+        for t0 in (0, 8128, 16384 - W // 2, T - W):
+            ref = op.project(x[b:b + 1, t0:t0 + W].float(), *weights, pos0=t0)
+            got = [o[b:b + 1, :, t0:t0 + W] for o in out]
+            compare(got, ref, f" (sequence {b}, tokens {t0}..{t0 + W - 1})")
