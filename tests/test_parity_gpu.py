@@ -422,6 +422,17 @@ def test_linear_decode_token_by_token_equals_forward_oracle(ttt):
     assert_close(out[2], bo, f, "b")
 
 
+def test_linear_decode_full_shape_one_token_per_call(ttt):
+    """The decode bench's launch: every (batch, head) stream of the 1.3B-layer
+    shape (B = 2, H = 32) decoded one token per call over three mini-batches,
+    outputs and both states against the oracle's decode of the same calls."""
+    w = WORKLOADS["decode_1p3b"].with_shape(T=48)
+    inp = make_inputs(w, 6)
+    cuts = list(range(1, 48))
+    compare_decode(gpu_decode_pieces(ttt, w, inp, cuts), oracle_decode_pieces(w, inp, cuts), TOL[w.dtype],
+                   w.mode == MODE_PLAIN)
+
+
 def test_linear_decode_one_call_is_the_generic_forward(ttt):
     """From a mini-batch boundary, one decode call at d = 32 (generic family)
     runs the generic forward scan operation for operation."""
@@ -559,6 +570,23 @@ def test_mlp_decode_pieces_vs_oracle(ttt, shape, mb, cuts, impl):
     inp = make_inputs(w, 3)
     out = gpu_mlp_decode_pieces(ttt, w, inp, cuts, mb, impl)
     ref = oracle_mlp_decode_pieces(w, inp, cuts, mb)
+    f = TOL[w.dtype]
+    assert_close(out[0], ref[0], f, "Z")
+    names = ("W1", "b1", "W2", "b2", "W1_mb", "b1_mb", "W2_mb", "b2_mb")
+    for name, o, r in zip(names, out[1:], ref[1:]):
+        scale = rms(r) if np.any(r) else 1.0
+        assert_close(o, r, f, name, denom=max(scale, 1e-3 * rms(ref[1])))
+
+
+def test_mlp_decode_full_shape_one_token_per_call(ttt):
+    """The TTT-MLP decode bench's launch (B = 4, H = 12, hidden 256) decoded one
+    token per call over two and a half mini-batches, outputs and both states
+    against the oracle's decode of the same calls."""
+    w = WORKLOADS["decode_mlp_8k"].with_shape(T=40)
+    inp = make_inputs(w, 7)
+    cuts = list(range(1, 40))
+    out = gpu_mlp_decode_pieces(ttt, w, inp, cuts, w.mini_batch)
+    ref = oracle_mlp_decode_pieces(w, inp, cuts, w.mini_batch)
     f = TOL[w.dtype]
     assert_close(out[0], ref[0], f, "Z")
     names = ("W1", "b1", "W2", "b2", "W1_mb", "b1_mb", "W2_mb", "b2_mb")
