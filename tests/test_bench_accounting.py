@@ -76,3 +76,24 @@ def test_recorded_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     assert bench.recorded_traffic(kernel, "linear_1p3b_32k") == 123
     assert bench.recorded_traffic(kernel, "linear_125m_2k") is None   # stale record
     assert bench.recorded_traffic(kernel, "mlp_8k") is None           # no record
+
+
+def test_committed_traffic_records_are_well_formed():
+    """Every line of the committed table names a kernel bench.py can hash and a
+    workload it runs, with a 16-digit hex hash and a positive byte count, and no
+    (kernel, workload) pair appears twice."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    seen = set()
+    with open(path) as fh:
+        for line in fh:
+            f = line.split("#")[0].split()
+            if not f:
+                continue
+            assert len(f) == 4, line
+            kernel, workload, digest, nbytes = f
+            assert kernel in bench.KERNEL_SOURCES, line
+            assert workload in WORKLOADS or workload in bench.PROLOGUES or workload in bench.BACKWARD, line
+            assert len(digest) == 16 and int(digest, 16) >= 0, line
+            assert int(nbytes) > 0, line
+            assert (kernel, workload) not in seen, line
+            seen.add((kernel, workload))
